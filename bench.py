@@ -1,0 +1,409 @@
+"""Benchmark of the H2O chunk step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+One step = one chunk of S query tokens through the whole path (attention with
+summed weights, score accumulate, select, scatter) on one layer's caches.  The
+default workload is the 2k-slot / 1k-chunk configuration (B=1, Hq=32, Hkv=8,
+d=128, M=2048, R=256, bf16).  Inputs are resident in HBM before timing; L2 is
+flushed (a 256 MiB write) between steps, outside the per-step CUDA events.  At
+N > 1 GPUs every rank runs an independent replica on its own seeded stream (the
+path has no cross-GPU exchange); the time is the max over ranks.
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the float64 CPU oracle
+instead, on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "H2O chunk-step query-tokens/s"
+UNIT = "query-tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def attn_pairs(cfg, S, n_valid):
+    """(query-head row, visible key) pairs of one step: B*Hq*(S*n_valid + S(S+1)/2)."""
+    return cfg.B * cfg.Hq * (S * n_valid + S * (S + 1) // 2)
+
+
+def select_scatter_bytes(cfg, S):
+    """Algorithmic bytes of score accumulate + select + scatter for one step:
+    scores and positions read and written once, the chunk's K/V rows read and
+    written once, the new scores written."""
+    BH = cfg.B * cfg.Hkv
+    es = 2 if cfg.dtype == torch.bfloat16 else 4
+    state = BH * cfg.M * (4 + 4) * 2
+    rows = BH * S * cfg.d * es * 2 * 2
+    return state + rows
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax = float(parts[1])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(cfg, chunks_host, budget_s, max_head_chunks=None):
+    """Times the float64 oracle on (batch 0, KV head h) caches, chunk after chunk,
+    until about budget_s seconds of step work are done.  Returns
+    (tokens/s extrapolated to the whole step, description, head-chunks timed)."""
+    from oracle import H2OHeadOracle
+    G = cfg.G
+    done, elapsed, heads_used = 0, 0.0, 0
+    for h in range(cfg.Hkv):
+        st = H2OHeadOracle(cfg.M, cfg.R, G, cfg.d)
+        q0, k0, v0 = chunks_host[0]
+        st.step(q0[0, h * G:(h + 1) * G], k0[0, h], v0[0, h])           # prefill, untimed
+        heads_used += 1
+        for (q, k, v) in chunks_host[1:]:
+            t = time.perf_counter()
+            st.step(q[0, h * G:(h + 1) * G], k[0, h], v[0, h])
+            elapsed += time.perf_counter() - t
+            done += 1
+            if elapsed >= budget_s or (max_head_chunks and done >= max_head_chunks):
+                break
+        if elapsed >= budget_s or (max_head_chunks and done >= max_head_chunks):
+            break
+    scale = cfg.B * cfg.Hkv * cfg.layers
+    per_step = elapsed / done * scale
+    rate = cfg.B * cfg.S / per_step
+    desc = (f"float64 oracle, {done} (KV head, chunk) steps of batch 0 over {heads_used} head(s) "
+            f"in {elapsed:.1f} s, extrapolated x{scale} (batch, layer, KV head) caches per step")
+    return rate, desc, done, elapsed
+
+
+def run_reference(args, cfg):
+    """--impl reference: the oracle as it stands, one (KV head, chunk) per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    import numpy as np
+    n_needed = args.warmup + args.steps
+    T = min(cfg.T, cfg.P + cfg.S * max(1, min(n_needed, cfg.n_chunks)))
+    Q, K, V = gen_batch(cfg, 0, device="cpu", T=T)
+    ch = [tuple(x.double().numpy() for x in c)
+          for c in split_chunks(Q[:1], K[:1], V[:1], [(a, b) for a, b in cfg.bounds() if a < T])]
+    from oracle import H2OHeadOracle
+    G = cfg.G
+    st = H2OHeadOracle(cfg.M, cfg.R, G, cfg.d)
+    q0, k0, v0 = ch[0]
+    st.step(q0[0, 0:G], k0[0, 0], v0[0, 0])
+    times = []
+    for i in range(n_needed):
+        q, k, v = ch[1 + i % (len(ch) - 1)]
+        t = time.perf_counter()
+        st.step(q[0, 0:G], k[0, 0], v[0, 0])
+        dt = time.perf_counter() - t
+        if i >= args.warmup:
+            times.append(dt)
+    per_step = statistics.mean(times) * cfg.B * cfg.Hkv * cfg.layers
+    value = cfg.B * cfg.S / per_step
+    cores = blas_threads()
+    sample = (f"each step: the float64 oracle on one (batch 0, KV head 0) cache for one chunk, "
+              f"scaled x{cfg.B * cfg.Hkv * cfg.layers} (batch, layer, KV head) caches to a whole step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"{cfg.name}: {cfg.describe()}", "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, cfg):
+    world, rank, local = dist_setup(args.gpus)
+    import h2o_kv_cache_b200 as h2o
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    dev = torch.device("cuda", local if world > 1 else 0)
+    n_needed = args.warmup + 2 * args.steps + 1     # device-timed steps, then host-buffer steps
+    n_chunks = min(cfg.n_chunks, n_needed)
+    T = cfg.P + cfg.S * n_chunks
+    bounds = [(a, b) for a, b in cfg.bounds() if a < T]
+    layers = []                                    # per layer: (cache, chunks)
+    for layer in range(cfg.layers):
+        # each replica (rank) has its own seeded streams
+        Q, K, V = gen_batch(cfg, layer + 1000 * rank, device=dev, T=T)
+        chunks = split_chunks(Q, K, V, bounds)
+        del Q, K, V
+        cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype, device=dev)
+        cache.prefill(*chunks[0], want_out=False)
+        layers.append((cache, chunks))
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(layers[0][1][1][0])
+    n_avail = len(bounds) - 1
+    ci = 0
+
+    def step_all(out_buf, host=None):
+        """One step: the next chunk through every layer's cache."""
+        nonlocal ci
+        for li, (cache, chunks) in enumerate(layers):
+            c = host[li] if host is not None else chunks[1 + ci % n_avail]
+            cache.step(*c, out=out_buf)
+        ci += 1
+
+    for _ in range(args.warmup):
+        step_all(out)
+    for cache, _ in layers:
+        cache.set_profiling(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    kern_ms = []
+    pairs = 0
+    launches = 0
+    barrier(world)
+    with ClockSampler(local if world > 1 else 0) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            for cache, _ in layers:
+                pairs += attn_pairs(cfg, cfg.S, cache.info()["n_valid"])
+            if len(layers) == 1:
+                ev[i][0].record(stream)
+                step_all(out)
+                ev[i][1].record(stream)
+                kern_ms.append(layers[0][0].last_timings())
+            else:
+                # per-layer timings need each layer's events read before its next step
+                ev[i][0].record(stream)
+                t = [0.0, 0.0, 0.0, 0.0]
+                for li, (cache, chunks) in enumerate(layers):
+                    cache.step(*chunks[1 + ci % n_avail], out=out)
+                    t = [a + b for a, b in zip(t, cache.last_timings())]
+                ci += 1
+                ev[i][1].record(stream)
+                kern_ms.append(t)
+            launches += sum(c.info()["launches"] for c, _ in layers)
+        barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_s = max_over_ranks(sum(step_ms) / 1e3, world)
+    value = world * cfg.B * cfg.S * args.steps / total_s
+    attn_ms = statistics.mean(k[0] for k in kern_ms) / cfg.layers
+    sel_ms = statistics.mean(k[1] + k[2] + k[3] for k in kern_ms) / cfg.layers
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the region
+    for cache, _ in layers:
+        cache.set_profiling(False)
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = d2h = 0
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    host_steps = []
+    for i in range(args.steps):
+        hs = []
+        for cache, chunks in layers:
+            q, k, v = chunks[1 + (ci + i) % n_avail]
+            hs.append(tuple(x.cpu().pin_memory() for x in (q, k, v)))
+        host_steps.append(hs)
+    h2d = sum(x.numel() * x.element_size() for hs in host_steps[0] for x in hs)
+    d2h = hout.numel() * hout.element_size() * len(layers)
+    barrier(world)
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        step_all(hout, host=host_steps[i])
+        e2e_ev[i][1].record(stream)
+    barrier(world)
+    e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3, world)
+    e2e_value = world * cfg.B * cfg.S * args.steps / e2e_s
+
+    peaks = load_peaks()
+    flops = 4 * cfg.d * pairs / (args.steps * cfg.layers)       # per attention launch
+    achieved_tflops = flops / (attn_ms * 1e-3) / 1e12
+    sel_bytes = select_scatter_bytes(cfg, cfg.S)
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tfile):
+        try:
+            with open(tfile) as f:
+                ent = json.load(f).get(cfg.name)
+            if ent and ent.get("lib_sha") == lib_sha():
+                traffic = ent["dram_bytes_per_launch"]
+        except (OSError, ValueError):
+            traffic = None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_s * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: {cfg.describe()}", "global_batch": cfg.B * world,
+                   "seq_len": cfg.S, "parallelism": f"replicas x{world}" if world > 1 else "single",
+                   "l2": "flushed between steps (256 MiB write outside the per-step events)"},
+        "roofline": {"bound": "tensor", "achieved": achieved_tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved_tflops / peaks["bf16_tflops"], "traffic": traffic,
+                     "kernel": "attention + summed weights",
+                     "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                     "algorithmic_flops_per_launch": flops, "ms_per_launch": attn_ms},
+        "roofline_select_scatter": {"bound": "hbm", "achieved": sel_bytes / (sel_ms * 1e-3) / 1e9,
+                                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": sel_bytes / (sel_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                    "algorithmic_bytes_per_launch_set": sel_bytes,
+                                    "ms_per_launch_set": sel_ms},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+        "kernel_ms_per_layer": {"attention": attn_ms,
+                                "score_reduce": statistics.mean(k[1] for k in kern_ms) / cfg.layers,
+                                "select": statistics.mean(k[2] for k in kern_ms) / cfg.layers,
+                                "scatter": statistics.mean(k[3] for k in kern_ms) / cfg.layers},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        chunks0 = layers[0][1]
+        chunks_host = [tuple(x[:1].double().cpu().numpy() for x in c) for c in chunks0[:8]]
+        rate, desc, n, el = oracle_sample(cfg, chunks_host, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(),
+                                "kind": "oracle", "sample": desc}
+    for cache, _ in layers:
+        cache.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def lib_sha():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "h2o_kv_cache_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from h2o_kv_cache_b200.workload import CONFIGS
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,167 @@
+"""H2O chunked sparse attention for B200 (sm_100a).
+
+A thin Python layer over libh2o.so (see include/h2o.h).  PyTorch supplies device
+memory and streams; every step of the chunk -- attention with summed weights,
+score accumulation, selection and scatter -- runs in the library's kernels.
+
+    cache = H2OCache(M=2048, R=256, Hq=32, Hkv=8, d=128, dtype=torch.bfloat16)
+    out = cache.prefill(q, k, v)          # q [B,Hq,P,d], k/v [B,Hkv,P,d]
+    out = cache.step(q, k, v)             # one chunk of S tokens
+    slots, scores, positions = cache.read_state()
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (H2O_BF16, H2O_F32, H2O_OK, STATUS_NAMES, lib)
+
+__all__ = ["H2OCache", "H2OError", "select", "lib"]
+
+_DTYPES = {torch.float32: H2O_F32, torch.bfloat16: H2O_BF16}
+
+
+class H2OError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _check(rc: int, handle=None):
+    if rc != H2O_OK:
+        raise H2OError(rc, lib.h2o_last_error(handle).decode())
+    return rc
+
+
+def _stream_ptr(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+class H2OCache:
+    """One layer's H2O caches for B sequences (batch fixed at prefill)."""
+
+    def __init__(self, M: int, R: int, Hq: int, Hkv: int, d: int, dtype=torch.bfloat16,
+                 device=None):
+        if dtype not in _DTYPES:
+            raise ValueError("dtype must be torch.float32 or torch.bfloat16")
+        self.M, self.R, self.Hq, self.Hkv, self.d, self.dtype = M, R, Hq, Hkv, d, dtype
+        self.device = torch.device(device if device is not None else "cuda", )
+        if self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
+        h = ctypes.c_void_p()
+        _check(lib.h2o_create(M, R, Hq, Hkv, d, _DTYPES[dtype], ctypes.byref(h)))
+        self._h = h
+        self.B = None
+        self.last_S = None
+
+    # -- helpers -------------------------------------------------------------
+    def _chk(self, rc):
+        return _check(rc, self._h)
+
+    def _args(self, q, k, v, S):
+        for name, t, H in (("q", q, self.Hq), ("k", k, self.Hkv), ("v", v, self.Hkv)):
+            if t.dtype != self.dtype or not t.is_contiguous() or t.dim() != 4:
+                raise ValueError(f"{name} must be a contiguous 4-d {self.dtype} tensor")
+            if t.shape[1] != H or t.shape[3] != self.d or t.shape[2] != S:
+                raise ValueError(f"{name} has shape {tuple(t.shape)}")
+        if k.shape != v.shape or k.shape[0] != q.shape[0]:
+            raise ValueError("q, k, v batch / shape mismatch")
+
+    def _out(self, q, out):
+        if out is None:
+            out = torch.empty_like(q)
+        elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+            raise ValueError("out must be contiguous, same shape and dtype as q")
+        return out
+
+    # -- API -----------------------------------------------------------------
+    def prefill(self, q, k, v, out=None, stream=None, want_out=True):
+        B, P = q.shape[0], q.shape[2]
+        self._args(q, k, v, P)
+        out = self._out(q, out) if want_out else None
+        with torch.cuda.device(self.device):
+            self._chk(lib.h2o_prefill(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, P,
+                                      _stream_ptr(stream, self.device)))
+        self.B, self.last_S = B, P
+        return out
+
+    def step(self, q, k, v, out=None, stream=None):
+        S = q.shape[2]
+        self._args(q, k, v, S)
+        out = self._out(q, out)
+        with torch.cuda.device(self.device):
+            self._chk(lib.h2o_step(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), S,
+                                   _stream_ptr(stream, self.device)))
+        self.last_S = S
+        return out
+
+    def read_state(self, stream=None):
+        """(slots [B,Hkv,S_last] int32, scores [B,Hkv,M] f32, positions [B,Hkv,M] int32)."""
+        dev = self.device
+        slots = torch.empty(self.B, self.Hkv, self.last_S, dtype=torch.int32, device=dev)
+        scores = torch.empty(self.B, self.Hkv, self.M, dtype=torch.float32, device=dev)
+        pos = torch.empty(self.B, self.Hkv, self.M, dtype=torch.int32, device=dev)
+        with torch.cuda.device(dev):
+            self._chk(lib.h2o_read_state(self._h, _ptr(slots), _ptr(scores), _ptr(pos),
+                                         _stream_ptr(stream, dev)))
+        return slots, scores, pos
+
+    def read_kv(self, stream=None):
+        shape = (self.B, self.Hkv, self.M, self.d)
+        kc = torch.empty(shape, dtype=self.dtype, device=self.device)
+        vc = torch.empty(shape, dtype=self.dtype, device=self.device)
+        with torch.cuda.device(self.device):
+            self._chk(lib.h2o_read_kv(self._h, _ptr(kc), _ptr(vc), _stream_ptr(stream, self.device)))
+        return kc, vc
+
+    def info(self):
+        arr = (ctypes.c_int64 * 5)()
+        self._chk(lib.h2o_info(self._h, arr))
+        return {"B": arr[0], "t0": arr[1], "n_valid": arr[2], "last_S": arr[3], "launches": arr[4]}
+
+    def set_profiling(self, on: bool):
+        self._chk(lib.h2o_set_profiling(self._h, 1 if on else 0))
+
+    def last_timings(self):
+        """ms of [attention, score accumulate, select, scatter] of the last step."""
+        arr = (ctypes.c_float * 4)()
+        n = lib.h2o_last_timings(self._h, arr, 4)
+        if n < 0:
+            self._chk(n)
+        return list(arr)[:n]
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib.h2o_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def select(scores, positions, t0: int, R: int, need: int, stream=None):
+    """Standalone selection: scores [n, M] f32, positions [n, M] int32 (device) ->
+    evicted [n, need] int32, ascending slots of the `need` smallest (score, pos)
+    among slots with 0 <= pos < t0 - R."""
+    n, M = scores.shape
+    if scores.dtype != torch.float32 or positions.dtype != torch.int32:
+        raise ValueError("scores must be float32 and positions int32")
+    if not scores.is_cuda or not positions.is_cuda:
+        raise ValueError("scores and positions must be CUDA tensors")
+    sc, ps = scores.contiguous(), positions.contiguous()     # kept alive across the call
+    ev = torch.empty(n, need, dtype=torch.int32, device=scores.device)
+    with torch.cuda.device(scores.device):
+        _check(lib.h2o_select(_ptr(sc), _ptr(ps), n, M, t0, R, need, _ptr(ev),
+                              _stream_ptr(stream, scores.device)))
+    return ev

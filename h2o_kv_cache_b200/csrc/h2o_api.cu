@@ -1,0 +1,456 @@
+// C ABI of the H2O chunk-step library: handle, device state, and the
+// stream-ordered sequence attend -> accumulate -> select -> scatter.
+// The operation each call performs is documented in include/h2o.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "../../include/h2o.h"
+#include "h2o_internal.cuh"
+
+namespace {
+
+thread_local std::string g_thread_err = "no error";
+
+struct DevBuf {
+  void* p = nullptr;
+  size_t cap = 0;
+};
+
+}  // namespace
+
+struct h2o_ctx {
+  int64_t M = 0, R = 0;
+  int Hq = 0, Hkv = 0, d = 0, dtype = 0, G = 0, esize = 0;
+  int B = 0;
+  int device = -1;
+  int64_t t0 = 0, n_valid = 0, last_S = 0;
+  int last_launches = 0;
+  bool prefilled = false;
+  bool use_umma = false;
+  int row_tile = h2o::kSimtRowTile;
+
+  // device state
+  void* kc = nullptr;
+  void* vc = nullptr;
+  float* scores = nullptr;
+  int32_t* pos = nullptr;
+  int* err = nullptr;
+  DevBuf partials, newscore, freed;
+  // staging for host pointers
+  DevBuf st_q, st_k, st_v, st_out;
+  int* h_err = nullptr;  // pinned mirror of *err
+  cudaEvent_t err_ev = nullptr;
+  bool err_pending = false;
+
+  bool prof = false;
+  cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  bool ev_valid = false;
+
+  std::string msg = "no error";
+};
+
+namespace {
+
+int fail(h2o_ctx* h, int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  if (h) h->msg = buf;
+  g_thread_err = buf;
+  return code;
+}
+
+int cuda_fail(h2o_ctx* h, cudaError_t e, const char* what) {
+  const int code = (e == cudaErrorMemoryAllocation) ? H2O_ENOMEM : H2O_ECUDA;
+  return fail(h, code, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define H2O_CUDA(h, call, what)                      \
+  do {                                               \
+    cudaError_t e_ = (call);                         \
+    if (e_ != cudaSuccess) return cuda_fail(h, e_, what); \
+  } while (0)
+
+bool fault_injected(const char* kind) {
+  const char* f = getenv("H2O_FAULT");
+  return f && strcmp(f, kind) == 0;
+}
+
+cudaError_t dev_alloc(void** p, size_t bytes) {
+  if (fault_injected("alloc")) return cudaErrorMemoryAllocation;
+  return cudaMalloc(p, bytes);
+}
+
+// Grow a scratch buffer (contents are not preserved).
+cudaError_t ensure(DevBuf& b, size_t bytes) {
+  if (b.cap >= bytes) return cudaSuccess;
+  if (b.p) {
+    cudaError_t e = cudaFree(b.p);
+    b.p = nullptr;
+    b.cap = 0;
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = dev_alloc(&b.p, bytes);
+  if (e == cudaSuccess) b.cap = bytes;
+  return e;
+}
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+bool sync_check_enabled() {
+  const char* s = getenv("H2O_SYNC_CHECK");
+  return s && s[0] == '1';
+}
+
+// Reads the device error word of a finished step; returns a status.
+int check_device_error(h2o_ctx* h, bool wait) {
+  if (!h->err_pending) return H2O_OK;
+  if (wait) {
+    cudaError_t e = cudaEventSynchronize(h->err_ev);
+    if (e != cudaSuccess) return cuda_fail(h, e, "kernel execution");
+  } else {
+    cudaError_t e = cudaEventQuery(h->err_ev);
+    if (e == cudaErrorNotReady) return H2O_OK;
+    if (e != cudaSuccess) return cuda_fail(h, e, "kernel execution");
+  }
+  h->err_pending = false;
+  const int w = *h->h_err;
+  if (w == 0) return H2O_OK;
+  // report once: clear the word so the handle's next step starts clean
+  *h->h_err = 0;
+  cudaMemset(h->err, 0, sizeof(int));
+  if (w & h2o::kErrTimeout)
+    return fail(h, H2O_ETIMEOUT, "a bounded in-kernel wait timed out (device error word 0x%x)", w);
+  if (w & h2o::kErrSelect)
+    return fail(h, H2O_ESHAPE, "fewer evictable slots than needed (device error word 0x%x)", w);
+  return fail(h, H2O_ECUDA, "device-side check failed (device error word 0x%x)", w);
+}
+
+size_t elem_size(int dtype) { return dtype == H2O_F32 ? 4 : 2; }
+
+// Runs one chunk of S tokens (prefill when the cache is empty).
+int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out, int64_t S,
+              cudaStream_t st) {
+  const int BH = h->B * h->Hkv;
+  const size_t es = elem_size(h->dtype);
+  const size_t q_bytes = (size_t)h->B * h->Hq * S * h->d * es;
+  const size_t kv_bytes = (size_t)BH * S * h->d * es;
+
+  int rc = check_device_error(h, sync_check_enabled());
+  if (rc != H2O_OK) return rc;
+
+  // need and eligibility are fixed by the bookkeeping: the min(R, t0) most
+  // recent tokens are always cached and protected, the rest of the valid slots
+  // are evictable.
+  const int64_t empties = h->M - h->n_valid;
+  const int64_t need = S > empties ? S - empties : 0;
+  const int64_t protect = h->R < h->t0 ? h->R : h->t0;
+  const int64_t eligible = h->n_valid - (protect < h->n_valid ? protect : h->n_valid);
+  if (need > eligible)
+    return fail(h, H2O_ESHAPE, "chunk of %lld tokens needs %lld evictions but only %lld slots are "
+                "older than the recent window", (long long)S, (long long)need, (long long)eligible);
+
+  // host-pointer staging
+  const void* dq = q;
+  const void* dk = k;
+  const void* dv = v;
+  void* dout = out;
+  const bool hq = !is_device_ptr(q), hk = !is_device_ptr(k), hv = !is_device_ptr(v);
+  const bool hout = out && !is_device_ptr(out);
+  if (hq) {
+    H2O_CUDA(h, ensure(h->st_q, q_bytes), "staging alloc");
+    H2O_CUDA(h, cudaMemcpyAsync(h->st_q.p, q, q_bytes, cudaMemcpyDefault, st), "copy q");
+    dq = h->st_q.p;
+  }
+  if (hk) {
+    H2O_CUDA(h, ensure(h->st_k, kv_bytes), "staging alloc");
+    H2O_CUDA(h, cudaMemcpyAsync(h->st_k.p, k, kv_bytes, cudaMemcpyDefault, st), "copy k");
+    dk = h->st_k.p;
+  }
+  if (hv) {
+    H2O_CUDA(h, ensure(h->st_v, kv_bytes), "staging alloc");
+    H2O_CUDA(h, cudaMemcpyAsync(h->st_v.p, v, kv_bytes, cudaMemcpyDefault, st), "copy v");
+    dv = h->st_v.p;
+  }
+  if (hout) {
+    H2O_CUDA(h, ensure(h->st_out, q_bytes), "staging alloc");
+    dout = h->st_out.p;
+  }
+
+  // scratch sized for this chunk
+  const int n_rt = (int)((S + h->row_tile - 1) / h->row_tile);
+  const size_t part_bytes = (size_t)BH * h->G * n_rt * (h->M + S) * sizeof(float);
+  H2O_CUDA(h, ensure(h->partials, part_bytes), "scratch alloc");
+  H2O_CUDA(h, ensure(h->newscore, (size_t)BH * S * sizeof(float)), "scratch alloc");
+  H2O_CUDA(h, ensure(h->freed, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
+
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(h->ev[0], st), "event");
+
+  h2o::AttnArgs a;
+  a.q = dq;
+  a.k = dk;
+  a.v = dv;
+  a.out = dout;
+  a.kc = h->kc;
+  a.vc = h->vc;
+  a.partials = static_cast<float*>(h->partials.p);
+  a.err = h->err;
+  a.B = h->B;
+  a.Hq = h->Hq;
+  a.Hkv = h->Hkv;
+  a.d = h->d;
+  a.S = S;
+  a.M = h->M;
+  a.n_valid = h->n_valid;
+  a.scale = (float)(1.0 / std::sqrt((double)h->d));
+  if (fault_injected("launch")) return fail(h, H2O_ECUDA, "injected launch failure");
+  cudaError_t e = h->use_umma ? h2o::launch_attn_umma(a, st) : h2o::launch_attn_simt(a, h->dtype, st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(h->ev[1], st), "event");
+
+  e = h2o::launch_score_reduce(static_cast<float*>(h->partials.p), h->scores,
+                               static_cast<float*>(h->newscore.p), BH, h->G, S, h->M,
+                               h->n_valid, h->row_tile, st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "score reduce launch");
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(h->ev[2], st), "event");
+
+  e = h2o::launch_select(h->scores, h->pos, BH, h->M, h->t0, h->R, need, h->n_valid, S,
+                         static_cast<int32_t*>(h->freed.p), S, h->err, st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "select launch");
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(h->ev[3], st), "event");
+
+  e = h2o::launch_scatter(dk, dv, h->kc, h->vc, h->scores, h->pos,
+                          static_cast<int32_t*>(h->freed.p), static_cast<float*>(h->newscore.p),
+                          BH, S, h->M, h->d, (int)es, h->t0, st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "scatter launch");
+  if (h->prof) {
+    H2O_CUDA(h, cudaEventRecord(h->ev[4], st), "event");
+    h->ev_valid = true;
+  }
+  h->last_launches = 4;
+
+  if (hout) H2O_CUDA(h, cudaMemcpyAsync(out, dout, q_bytes, cudaMemcpyDefault, st), "copy out");
+
+  // error word: async read-back, checked by the next call
+  H2O_CUDA(h, cudaMemcpyAsync(h->h_err, h->err, sizeof(int), cudaMemcpyDeviceToHost, st), "err copy");
+  H2O_CUDA(h, cudaEventRecord(h->err_ev, st), "event");
+  h->err_pending = true;
+
+  h->t0 += S;
+  h->n_valid = h->n_valid + S < h->M ? h->n_valid + S : h->M;
+  h->last_S = S;
+  if (hq || hk || hv || hout || sync_check_enabled()) {
+    rc = check_device_error(h, true);
+    if (rc != H2O_OK) return rc;
+  }
+  return H2O_OK;
+}
+
+int alloc_state(h2o_ctx* h, int B) {
+  const size_t es = elem_size(h->dtype);
+  const size_t slots = (size_t)B * h->Hkv * h->M;
+  H2O_CUDA(h, cudaGetDevice(&h->device), "cudaGetDevice");
+  H2O_CUDA(h, dev_alloc(&h->kc, slots * h->d * es), "cache alloc");
+  H2O_CUDA(h, dev_alloc(&h->vc, slots * h->d * es), "cache alloc");
+  H2O_CUDA(h, dev_alloc((void**)&h->scores, slots * sizeof(float)), "state alloc");
+  H2O_CUDA(h, dev_alloc((void**)&h->pos, slots * sizeof(int32_t)), "state alloc");
+  H2O_CUDA(h, dev_alloc((void**)&h->err, sizeof(int)), "state alloc");
+  H2O_CUDA(h, cudaMemset(h->kc, 0, slots * h->d * es), "memset");
+  H2O_CUDA(h, cudaMemset(h->vc, 0, slots * h->d * es), "memset");
+  H2O_CUDA(h, cudaMemset(h->scores, 0, slots * sizeof(float)), "memset");
+  H2O_CUDA(h, cudaMemset(h->pos, 0xFF, slots * sizeof(int32_t)), "memset");
+  H2O_CUDA(h, cudaMemset(h->err, 0, sizeof(int)), "memset");
+  H2O_CUDA(h, cudaMallocHost((void**)&h->h_err, sizeof(int)), "pinned alloc");
+  *h->h_err = 0;
+  H2O_CUDA(h, cudaEventCreateWithFlags(&h->err_ev, cudaEventDisableTiming), "event");
+  for (auto& ev : h->ev) H2O_CUDA(h, cudaEventCreate(&ev), "event");
+  H2O_CUDA(h, cudaDeviceSynchronize(), "state init");
+  h->B = B;
+  return H2O_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int h2o_create(int64_t M, int64_t R, int Hq, int Hkv, int d, int dtype, h2o_t* out) {
+  if (!out) return fail(nullptr, H2O_EINVAL, "h2o_create: out is NULL");
+  *out = nullptr;
+  if (M < 1 || R < 0 || R >= M)
+    return fail(nullptr, H2O_EINVAL, "h2o_create: need M >= 1 and 0 <= R < M (M=%lld R=%lld)",
+                (long long)M, (long long)R);
+  if (M > (int64_t)1 << 30)
+    return fail(nullptr, H2O_EINVAL, "h2o_create: M=%lld too large", (long long)M);
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
+    return fail(nullptr, H2O_EINVAL, "h2o_create: need Hq %% Hkv == 0 (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (d != 64 && d != 128) return fail(nullptr, H2O_EINVAL, "h2o_create: d must be 64 or 128 (d=%d)", d);
+  if (dtype != H2O_F32 && dtype != H2O_BF16)
+    return fail(nullptr, H2O_EINVAL, "h2o_create: dtype must be H2O_F32 or H2O_BF16");
+  h2o_ctx* h = new (std::nothrow) h2o_ctx();
+  if (!h) return fail(nullptr, H2O_ENOMEM, "h2o_create: out of host memory");
+  h->M = M;
+  h->R = R;
+  h->Hq = Hq;
+  h->Hkv = Hkv;
+  h->G = Hq / Hkv;
+  h->d = d;
+  h->dtype = dtype;
+  h->esize = (int)elem_size(dtype);
+  h->use_umma = h2o::attn_umma_supported(dtype, d);
+  h->row_tile = h->use_umma ? h2o::kUmmaRowTile : h2o::kSimtRowTile;
+  *out = h;
+  return H2O_OK;
+}
+
+int h2o_prefill(h2o_t h, const void* q, const void* k, const void* v, void* out, int B, int64_t P,
+                void* stream) {
+  if (!h) return fail(nullptr, H2O_EINVAL, "h2o_prefill: NULL handle");
+  if (h->prefilled) return fail(h, H2O_ESTATE, "h2o_prefill: handle already prefilled");
+  if (!q || !k || !v) return fail(h, H2O_EINVAL, "h2o_prefill: q, k and v must not be NULL");
+  if (B < 1 || P < 1) return fail(h, H2O_EINVAL, "h2o_prefill: need B >= 1 and P >= 1");
+  if (P > h->M)
+    return fail(h, H2O_ESHAPE, "h2o_prefill: P=%lld exceeds the cache capacity M=%lld",
+                (long long)P, (long long)h->M);
+  int rc = alloc_state(h, B);
+  if (rc != H2O_OK) return rc;
+  h->prefilled = true;
+  return run_chunk(h, q, k, v, out, P, static_cast<cudaStream_t>(stream));
+}
+
+int h2o_step(h2o_t h, const void* q, const void* k, const void* v, void* out, int64_t S,
+             void* stream) {
+  if (!h) return fail(nullptr, H2O_EINVAL, "h2o_step: NULL handle");
+  if (!h->prefilled) return fail(h, H2O_ESTATE, "h2o_step: called before h2o_prefill");
+  if (!q || !k || !v) return fail(h, H2O_EINVAL, "h2o_step: q, k and v must not be NULL");
+  if (S < 1) return fail(h, H2O_EINVAL, "h2o_step: need S >= 1");
+  if (S > h->M)
+    return fail(h, H2O_ESHAPE, "h2o_step: S=%lld exceeds the cache capacity M=%lld",
+                (long long)S, (long long)h->M);
+  return run_chunk(h, q, k, v, out, S, static_cast<cudaStream_t>(stream));
+}
+
+int h2o_read_state(h2o_t h, int32_t* slots, float* scores, int32_t* positions, void* stream) {
+  if (!h) return fail(nullptr, H2O_EINVAL, "h2o_read_state: NULL handle");
+  if (!h->prefilled) return fail(h, H2O_ESTATE, "h2o_read_state: called before h2o_prefill");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t slots_n = (size_t)h->B * h->Hkv * h->M;
+  if (slots)
+    H2O_CUDA(h, cudaMemcpyAsync(slots, h->freed.p, (size_t)h->B * h->Hkv * h->last_S * sizeof(int32_t),
+                                cudaMemcpyDefault, st), "copy slots");
+  if (scores)
+    H2O_CUDA(h, cudaMemcpyAsync(scores, h->scores, slots_n * sizeof(float), cudaMemcpyDefault, st),
+             "copy scores");
+  if (positions)
+    H2O_CUDA(h, cudaMemcpyAsync(positions, h->pos, slots_n * sizeof(int32_t), cudaMemcpyDefault, st),
+             "copy positions");
+  if ((slots && !is_device_ptr(slots)) || (scores && !is_device_ptr(scores)) ||
+      (positions && !is_device_ptr(positions))) {
+    H2O_CUDA(h, cudaStreamSynchronize(st), "read_state sync");
+    return check_device_error(h, true);
+  }
+  return check_device_error(h, false);
+}
+
+int h2o_read_kv(h2o_t h, void* k_cache, void* v_cache, void* stream) {
+  if (!h) return fail(nullptr, H2O_EINVAL, "h2o_read_kv: NULL handle");
+  if (!h->prefilled) return fail(h, H2O_ESTATE, "h2o_read_kv: called before h2o_prefill");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)h->B * h->Hkv * h->M * h->d * h->esize;
+  if (k_cache) H2O_CUDA(h, cudaMemcpyAsync(k_cache, h->kc, bytes, cudaMemcpyDefault, st), "copy k");
+  if (v_cache) H2O_CUDA(h, cudaMemcpyAsync(v_cache, h->vc, bytes, cudaMemcpyDefault, st), "copy v");
+  if ((k_cache && !is_device_ptr(k_cache)) || (v_cache && !is_device_ptr(v_cache)))
+    H2O_CUDA(h, cudaStreamSynchronize(st), "read_kv sync");
+  return H2O_OK;
+}
+
+int h2o_info(h2o_t h, int64_t out[5]) {
+  if (!h || !out) return fail(h, H2O_EINVAL, "h2o_info: NULL argument");
+  out[0] = h->B;
+  out[1] = h->t0;
+  out[2] = h->n_valid;
+  out[3] = h->last_S;
+  out[4] = h->last_launches;
+  return H2O_OK;
+}
+
+int h2o_set_profiling(h2o_t h, int on) {
+  if (!h) return fail(nullptr, H2O_EINVAL, "h2o_set_profiling: NULL handle");
+  if (on && !h->prefilled) return fail(h, H2O_ESTATE, "h2o_set_profiling: prefill first");
+  h->prof = on != 0;
+  h->ev_valid = false;
+  return H2O_OK;
+}
+
+int h2o_last_timings(h2o_t h, float* ms, int n) {
+  if (!h || (!ms && n > 0)) return fail(h, H2O_EINVAL, "h2o_last_timings: NULL argument");
+  if (!h->ev_valid) return fail(h, H2O_ESTATE, "h2o_last_timings: no profiled step");
+  H2O_CUDA(h, cudaEventSynchronize(h->ev[4]), "event sync");
+  int w = 0;
+  for (int i = 0; i < 4 && w < n; ++i, ++w)
+    H2O_CUDA(h, cudaEventElapsedTime(&ms[i], h->ev[i], h->ev[i + 1]), "event time");
+  return w;
+}
+
+int h2o_destroy(h2o_t h) {
+  if (!h) return H2O_OK;
+  if (h->device >= 0) {
+    cudaSetDevice(h->device);
+    cudaDeviceSynchronize();
+  }
+  cudaFree(h->kc);
+  cudaFree(h->vc);
+  cudaFree(h->scores);
+  cudaFree(h->pos);
+  cudaFree(h->err);
+  for (DevBuf* b : {&h->partials, &h->newscore, &h->freed, &h->st_q, &h->st_k, &h->st_v, &h->st_out})
+    cudaFree(b->p);
+  if (h->h_err) cudaFreeHost(h->h_err);
+  if (h->err_ev) cudaEventDestroy(h->err_ev);
+  for (auto ev : h->ev)
+    if (ev) cudaEventDestroy(ev);
+  delete h;
+  return H2O_OK;
+}
+
+const char* h2o_last_error(h2o_t h) { return h ? h->msg.c_str() : g_thread_err.c_str(); }
+
+int h2o_select(const float* scores, const int32_t* positions, int n_heads, int64_t M, int64_t t0,
+               int64_t R, int64_t need, int32_t* evicted, void* stream) {
+  if (!scores || !positions || (!evicted && need > 0))
+    return fail(nullptr, H2O_EINVAL, "h2o_select: NULL argument");
+  if (n_heads < 1 || M < 1 || need < 0 || need > M || R < 0)
+    return fail(nullptr, H2O_EINVAL, "h2o_select: bad sizes");
+  if (need == 0) return H2O_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* derr = nullptr;
+  cudaError_t e = cudaMallocAsync((void**)&derr, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(nullptr, e, "h2o_select: alloc");
+  cudaMemsetAsync(derr, 0, sizeof(int), st);
+  // the kernel writes `need` evictions then S - need "empty" slots; S = need here
+  e = h2o::launch_select(scores, positions, n_heads, M, t0, R, need, M, need, evicted, need, derr, st);
+  int hv = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&hv, derr, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  cudaFreeAsync(derr, st);
+  if (e != cudaSuccess) return cuda_fail(nullptr, e, "h2o_select");
+  if (hv & h2o::kErrSelect) return fail(nullptr, H2O_ESHAPE, "h2o_select: fewer eligible slots than need");
+  return H2O_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,150 @@
+/*
+ * h2o.h -- C ABI of the H2O chunk-step library (libh2o.so, sm_100a).
+ *
+ * Method: H2O (heavy-hitter oracle) sparse attention over a fixed-capacity KV
+ * cache, processed chunk by chunk, as described in "Learning how to Forget:
+ * Fine-tuning for Long-Context Sparse Attention":
+ *   - Abstract: an implementation of H2O sparse attention with a dedicated
+ *     scaled dot product attention (SDPA) kernel;
+ *   - §1 Introduction ¶1: KV information is held in a fixed-size cache whose
+ *     slots are evicted once it is full;
+ *   - §1 Introduction ¶3: combinable with grouped query attention (GQA);
+ *   - FAQ answer 3: the SDPA kernel also returns the summed attention weights;
+ *   - Figure 1(a): a prefill chunk of full length, then chunks of S tokens.
+ *
+ * One chunk step, per (batch b, KV head h), with t0 = tokens already seen:
+ *   1. attend:  each query row (g, i) of h's group (query head g uses KV head
+ *               g / (Hq/Hkv)) sees every valid cache slot plus the chunk keys
+ *               j <= i; p = softmax(q.k / sqrt(d)); out = p . V.
+ *   2. summed weights: c_j = sum over the group's query heads and the chunk's
+ *               queries of p_ij, for each cache slot and each chunk key.
+ *   3. accumulate: score[slot] += c_slot for every valid slot (running sum).
+ *   4. evict:   need = max(0, S - empty slots); among valid slots whose token
+ *               position is older than the recent window (pos < t0 - R), the
+ *               `need` smallest by (score, pos) are evicted.
+ *   5. scatter: freed = ascending(evicted slots, then the first S - need empty
+ *               slots); chunk token i goes to freed[i]: its K and V rows,
+ *               pos = t0 + i, score = c of chunk key i.
+ * A prefill is the same step on an empty cache (it evicts nothing).
+ *
+ * Layouts (row-major, contiguous, element type = the handle's dtype):
+ *   q, out        [B, Hq,  S, d]
+ *   k, v          [B, Hkv, S, d]
+ *   cache K, V    [B, Hkv, M, d]   (library-owned)
+ *   scores        [B, Hkv, M]  float32;  positions [B, Hkv, M] int32 (-1 = empty)
+ *
+ * Pointers: q/k/v/out and every read-back buffer may be device memory or host
+ * memory (pinned or pageable); host buffers are staged through library-owned
+ * device buffers with stream-ordered copies.  The caller owns all of them.
+ * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream); every
+ * call only enqueues work on it, except where stated.  A handle is not
+ * thread-safe.
+ *
+ * Errors: every call returns an h2o_status; nothing aborts or throws across the
+ * ABI.  h2o_last_error() gives the message of the last failing call.  A device
+ * error raised by an earlier step (e.g. a bounded wait that timed out inside a
+ * kernel) is reported by the next call on the handle as H2O_ETIMEOUT or
+ * H2O_ECUDA.
+ */
+#ifndef H2O_H_
+#define H2O_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct h2o_ctx* h2o_t;
+
+typedef enum {
+  H2O_OK = 0,
+  H2O_EINVAL = -1,   /* bad argument (null pointer, dtype, d, Hq % Hkv, R >= M) */
+  H2O_ESHAPE = -2,   /* shape cannot be served: P > M, S > M, or fewer evictable slots than needed */
+  H2O_ESTATE = -3,   /* step before prefill, prefill twice */
+  H2O_ENOMEM = -4,   /* a device or pinned allocation failed */
+  H2O_ECUDA = -5,    /* a CUDA runtime call or kernel launch failed */
+  H2O_ETIMEOUT = -6  /* a bounded in-kernel wait ran out; the step's results are invalid */
+} h2o_status;
+
+typedef enum { H2O_F32 = 0, H2O_BF16 = 1 } h2o_dtype;
+
+/* Create a handle for one layer's caches.
+ *   M    cache capacity (slots) per (batch, KV head), M >= 1
+ *   R    protected recent window in tokens, 0 <= R < M
+ *   Hq   query heads; Hkv KV heads; Hq % Hkv == 0
+ *   d    head dimension, 64 or 128
+ *   dtype H2O_F32 or H2O_BF16 (q/k/v/out/cache element type)
+ * No device memory is allocated until the prefill (the batch size is known
+ * then).  The scale is fixed at 1/sqrt(d); natural-base softmax.
+ * Returns H2O_OK and *out, or H2O_EINVAL.                                     */
+int h2o_create(int64_t M, int64_t R, int Hq, int Hkv, int d, int dtype, h2o_t* out);
+
+/* Prefill: the first chunk, P tokens (1 <= P <= M), causal attention among
+ * themselves with an empty cache.  Token t goes to slot t with score = its
+ * summed attention weight.  Allocates the cache (zero-filled), scores,
+ * positions and scratch on the current device.  `out` may be NULL (outputs
+ * are then not written).  Errors: H2O_ESTATE if already prefilled, H2O_ESHAPE
+ * if P > M, H2O_ENOMEM.                                                       */
+int h2o_prefill(h2o_t h, const void* q, const void* k, const void* v, void* out,
+                int B, int64_t P, void* stream);
+
+/* One chunk step of S tokens (1 <= S <= M) at t0 = tokens seen so far, on the
+ * batch size fixed at prefill: attend, accumulate, evict, scatter (see top).
+ * The new K/V rows are copied into the cache inside the step, so the caller
+ * may reuse q/k/v once the stream has passed the step.
+ * Errors: H2O_ESTATE before prefill; H2O_ESHAPE if fewer than `need` slots are
+ * evictable (valid slots minus the min(R, t0) protected ones).                */
+int h2o_step(h2o_t h, const void* q, const void* k, const void* v, void* out,
+             int64_t S, void* stream);
+
+/* Copy the state out (each pointer may be NULL to skip it):
+ *   slots      [B, Hkv, S_last] int32: the slots the last step (or prefill)
+ *              filled, ascending; these are its evicted slots followed by the
+ *              previously empty slots it used
+ *   scores     [B, Hkv, M] float32 (0 for empty slots)
+ *   positions  [B, Hkv, M] int32, -1 for empty slots
+ * Errors: H2O_ESTATE before prefill.                                          */
+int h2o_read_state(h2o_t h, int32_t* slots, float* scores, int32_t* positions, void* stream);
+
+/* Copy the cache contents out: k_cache, v_cache [B, Hkv, M, d] of the handle's
+ * dtype (NULL skips).  Rows of empty slots are zero.                          */
+int h2o_read_kv(h2o_t h, void* k_cache, void* v_cache, void* stream);
+
+/* Counters of the handle: out[0] = B, out[1] = t0 (tokens seen), out[2] =
+ * valid slots per (batch, KV head), out[3] = S of the last step, out[4] =
+ * device kernels launched by the last step (or prefill).                      */
+int h2o_info(h2o_t h, int64_t out[5]);
+
+/* Per-kernel timing.  When on (default off), each step records CUDA events
+ * around its kernels on the caller's stream; h2o_last_timings() waits for the
+ * last step's events and writes up to n durations in milliseconds:
+ *   ms[0] attention + summed weights, ms[1] score accumulate, ms[2] select,
+ *   ms[3] scatter.  Returns the number written (>= 0) or a negative status. */
+int h2o_set_profiling(h2o_t h, int on);
+int h2o_last_timings(h2o_t h, float* ms, int n);
+
+/* Free every resource of the handle (synchronises the device first).  NULL is
+ * accepted.                                                                   */
+int h2o_destroy(h2o_t h);
+
+/* Message of the last failing call on h (or of the last failing h2o_create /
+ * standalone call on this thread when h is NULL).  Never NULL.                */
+const char* h2o_last_error(h2o_t h);
+
+/* Standalone selection step (step 4 above) on caller-owned device arrays, for
+ * n_heads independent caches of M slots each:
+ *   scores [n_heads, M] float32, positions [n_heads, M] int32 (-1 = empty)
+ *   evicted [n_heads, need] int32 (output): the `need` smallest (score, pos)
+ *   among slots with 0 <= pos < t0 - R, ascending by slot.
+ * Errors: H2O_EINVAL on bad sizes; H2O_ESHAPE if a cache has fewer than `need`
+ * eligible slots (checked on the device; reported by this call, which then
+ * synchronises the stream).                                                   */
+int h2o_select(const float* scores, const int32_t* positions, int n_heads, int64_t M,
+               int64_t t0, int64_t R, int64_t need, int32_t* evicted, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H2O_H_ */

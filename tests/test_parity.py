@@ -1,0 +1,261 @@
+"""GPU path vs the float64 oracle, through the C ABI (needs a B200).
+
+Every chunk of a seeded stream runs on the GPU (prefill, then steps) and in the
+oracle on the same input values; outputs, scores, evictions, slot -> position
+maps and the cache's K/V bytes are compared with the tolerances of
+tests/parity_util.py.  Small configurations run the oracle on every head and
+every chunk; the full-size workloads run it on sampled (batch, KV head) caches
+-- either along the whole stream, or on sampled chunks after loading the GPU's
+state into the oracle.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import H2OHeadOracle, H2OOracle, select_evictions
+from tests.parity_util import (annotate_boundary, check_evictions, check_outputs, check_scores,
+                               to64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def h2o(cuda_ok):
+    import h2o_kv_cache_b200 as m
+    return m
+
+
+def _cfg(base, **kw):
+    from h2o_kv_cache_b200.workload import CONFIGS
+    return dataclasses.replace(CONFIGS[base] if isinstance(base, int) else base, **kw)
+
+
+def _sync_head(st, kc, vc, scores, pos, b, h, t0):
+    st.load_state(to64(kc[b, h]), to64(vc[b, h]), scores[b, h], pos[b, h], t0)
+
+
+def run_stream(h2o, cfg, heads=None, layer=0, T=None, oracle_chunks=None, kv_check=True):
+    """Returns a summary dict.  oracle_chunks=None: the oracle follows the whole
+    stream; otherwise only the listed chunk indices are checked, each after
+    loading the GPU's pre-step state into the oracle."""
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    T = cfg.T if T is None else T
+    Q, K, V = gen_batch(cfg, layer, device="cuda", T=T)
+    bounds = [(a, b) for a, b in cfg.bounds() if a < T]
+    bounds[-1] = (bounds[-1][0], min(bounds[-1][1], T))
+    chunks = split_chunks(Q, K, V, bounds)
+    cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    G = cfg.G
+    if heads is None:
+        heads = [(b, h) for b in range(cfg.B) for h in range(cfg.Hkv)]
+    orc = {bh: H2OHeadOracle(cfg.M, cfg.R, G, cfg.d) for bh in heads}
+    Kn, Vn = to64(K), to64(V)
+    summary = {"chunks": 0, "ties": 0, "max_abs": 0.0, "rel_norm": 0.0, "score_rel": 0.0}
+    for ci, (q, k, v) in enumerate(chunks):
+        t0 = bounds[ci][0]
+        follow = oracle_chunks is None or ci in oracle_chunks
+        if follow and oracle_chunks is not None and ci > 0:
+            _, sc0, ps0 = cache.read_state()
+            kc0, vc0 = cache.read_kv()
+            sc0, ps0 = sc0.cpu().numpy(), ps0.cpu().numpy()
+            for (b, h), st in orc.items():
+                _sync_head(st, kc0, vc0, sc0, ps0, b, h, t0)
+        pos_before = {bh: st.pos.copy() for bh, st in orc.items()}
+        out = cache.prefill(q, k, v) if ci == 0 else cache.step(q, k, v)
+        torch.cuda.synchronize()
+        if not follow:
+            continue
+        slots, scores, pos = (x.cpu().numpy() for x in cache.read_state())
+        out64 = to64(out)
+        qn = to64(q)
+        kn_, vn_ = to64(k), to64(v)
+        kc = vc = None
+        for (b, h), st in orc.items():
+            gq = slice(h * G, (h + 1) * G)
+            ref = st.step(qn[b, gq], kn_[b, h], vn_[b, h])
+            where = f"{cfg.name} chunk {ci} (b={b}, h={h})"
+            r = check_outputs(out64[b, gq], ref, cfg.dtype, where)
+            summary["max_abs"] = max(summary["max_abs"], r["max_abs"])
+            summary["rel_norm"] = max(summary["rel_norm"], r["rel_norm"])
+            annotate_boundary(st, pos_before[(b, h)])
+            status = check_evictions(st, slots[b, h], where)
+            if status == "exact":
+                assert np.array_equal(pos[b, h], st.pos), f"{where}: slot -> position map differs"
+                summary["score_rel"] = max(summary["score_rel"],
+                                           check_scores(scores[b, h], st.score, st.pos >= 0, where))
+            else:
+                summary["ties"] += 1
+                # compare by position on the tokens both kept, then adopt the GPU state
+                gmap = {int(p): s for p, s in zip(pos[b, h], scores[b, h]) if p >= 0}
+                omap = {int(p): s for p, s in zip(st.pos, st.score) if p >= 0}
+                common = sorted(set(gmap) & set(omap))
+                check_scores(np.array([gmap[p] for p in common]), np.array([omap[p] for p in common]),
+                             np.ones(len(common), bool), where)
+                if kc is None:
+                    kc, vc = cache.read_kv()
+                _sync_head(st, kc, vc, scores, pos, b, h, t0 + (bounds[ci][1] - bounds[ci][0]))
+            if kv_check:
+                if kc is None:
+                    kc, vc = cache.read_kv()
+                valid = pos[b, h] >= 0
+                p = pos[b, h][valid]
+                assert torch.equal(kc[b, h][torch.from_numpy(valid).cuda()], K[b, h, torch.from_numpy(p).long().cuda()]), f"{where}: cached K rows differ from the stream"
+                assert torch.equal(vc[b, h][torch.from_numpy(valid).cuda()], V[b, h, torch.from_numpy(p).long().cuda()]), f"{where}: cached V rows differ from the stream"
+        summary["chunks"] += 1
+    info = cache.info()
+    assert info["t0"] == bounds[-1][1]
+    cache.close()
+    return summary
+
+
+# --------------------------------------------------------------------------------------
+# Small configurations: every head, every chunk
+# --------------------------------------------------------------------------------------
+def test_tiny_fp32_full_stream(h2o):
+    s = run_stream(h2o, _cfg(0))
+    assert s["chunks"] == 5
+
+
+def test_exact_attention_when_cache_never_fills(h2o):
+    cfg = _cfg(0, M=384, name="tiny-fp32-never-full")
+    s = run_stream(h2o, cfg)
+    assert s["ties"] == 0
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.float32, 128),
+                                     (torch.bfloat16, 64), (torch.bfloat16, 128)])
+def test_ragged_shapes(h2o, dtype, d):
+    # ragged prefill (partly full cache), ragged chunks, a ragged last chunk, B > 1
+    cfg = _cfg(0, name=f"ragged-{dtype}-{d}", B=2, Hq=6, Hkv=2, d=d, M=300, R=17, T=100 + 37 * 7 + 11,
+               P=100, S=37, dtype=dtype, planted=0.02)
+    run_stream(h2o, cfg)
+
+
+def test_large_gqa_group_and_long_tile_rows(h2o):
+    cfg = _cfg(0, name="gqa8-bf16", B=1, Hq=8, Hkv=1, d=128, M=520, R=40, T=520 + 3 * 260, P=520,
+               S=260, dtype=torch.bfloat16, planted=0.01)
+    run_stream(h2o, cfg)
+
+
+def test_single_token_steps_and_single_token_prefill(h2o):
+    cfg = _cfg(0, name="decode-like", M=40, R=4, T=1 + 70, P=1, S=1, planted=0.0)
+    run_stream(h2o, cfg)
+    cfg = _cfg(0, name="decode-bf16", M=72, R=5, T=72 + 30, P=72, S=1, dtype=torch.bfloat16, d=128)
+    run_stream(h2o, cfg)
+
+
+def test_window_just_below_capacity(h2o):
+    # R = M - S: exactly `need` slots are evictable at every step
+    cfg = _cfg(0, name="tight-window", M=96, R=64, T=96 + 32 * 5, P=96, S=32)
+    run_stream(h2o, cfg)
+
+
+# --------------------------------------------------------------------------------------
+# The benchmark workloads at full size
+# --------------------------------------------------------------------------------------
+def test_m2k_s1k_full_stream(h2o):
+    s = run_stream(h2o, _cfg(1))
+    assert s["chunks"] == 15
+
+
+def test_m16k_s1k_sampled_head_full_stream(h2o):
+    run_stream(h2o, _cfg(2), heads=[(0, 3)], kv_check=False)
+
+
+def test_m32k_s2k_sampled_chunks(h2o):
+    run_stream(h2o, _cfg(3), heads=[(0, 5)], oracle_chunks={1, 2, 48})
+
+
+def test_b4_layers_sampled_heads(h2o):
+    cfg = _cfg(4)
+    run_stream(h2o, cfg, heads=[(2, 6)], layer=0, kv_check=False)
+    run_stream(h2o, cfg, heads=[(1, 1)], layer=27, oracle_chunks={1, 24}, kv_check=False)
+
+
+# --------------------------------------------------------------------------------------
+# Prefill mass invariant at full size, errors, host pointers, standalone selection
+# --------------------------------------------------------------------------------------
+def test_prefill_mass_invariant_full_size(h2o):
+    from h2o_kv_cache_b200.workload import gen_batch
+    cfg = _cfg(3)
+    Q, K, V = gen_batch(cfg, 0, device="cuda", T=cfg.P)
+    cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    cache.prefill(Q, K, V)
+    _, scores, pos = cache.read_state()
+    tot = scores.double().sum(dim=2)
+    torch.testing.assert_close(tot, torch.full_like(tot, cfg.P * cfg.G), rtol=1e-4, atol=0)
+    assert torch.equal(pos[0, 0], torch.arange(cfg.P, dtype=torch.int32, device="cuda"))
+    cache.close()
+
+
+def test_shape_error_leaves_state_intact(h2o):
+    from h2o_kv_cache_b200.workload import gen_batch
+    cfg = _cfg(0, M=64, R=60, T=64 + 8, P=64, S=8)
+    Q, K, V = gen_batch(cfg, 0, device="cuda")
+    cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    cache.prefill(Q[:, :, :64].contiguous(), K[:, :, :64].contiguous(), V[:, :, :64].contiguous())
+    before = [x.clone() for x in cache.read_state()[1:]]
+    with pytest.raises(h2o.H2OError) as ei:    # 64 valid, min(R, t0) = 60 protected, need 8
+        cache.step(Q[:, :, 64:].contiguous(), K[:, :, 64:].contiguous(), V[:, :, 64:].contiguous())
+    assert ei.value.status == -2
+    after = cache.read_state()[1:]
+    assert all(torch.equal(a, b) for a, b in zip(before, after))
+    assert cache.info()["t0"] == 64
+    cache.close()
+
+
+def test_host_buffers_match_device_buffers(h2o):
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    cfg = _cfg(0, dtype=torch.bfloat16, d=128)
+    Q, K, V = gen_batch(cfg, 0, device="cuda")
+    chunks = split_chunks(Q, K, V, cfg.bounds())
+    a = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    b = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    for ci, (q, k, v) in enumerate(chunks):
+        pin = ci % 2 == 0
+        hq, hk, hv = (x.cpu().pin_memory() if pin else x.cpu() for x in (q, k, v))
+        hout = torch.empty_like(hq).pin_memory() if pin else torch.empty_like(hq)
+        oa = a.prefill(q, k, v) if ci == 0 else a.step(q, k, v)
+        ob = b.prefill(hq, hk, hv, out=hout) if ci == 0 else b.step(hq, hk, hv, out=hout)
+        torch.cuda.synchronize()
+        assert torch.equal(oa.cpu(), ob)
+    for x, y in zip(a.read_state(), b.read_state()):
+        assert torch.equal(x, y)
+    a.close()
+    b.close()
+
+
+def test_standalone_select_with_ties(h2o):
+    rng = np.random.default_rng(11)
+    for trial in range(12):
+        n, M = 3, int(rng.integers(8, 5000))
+        t0 = 10 * M
+        R = int(rng.integers(0, M // 2))
+        pos = np.stack([rng.permutation(t0)[:M] for _ in range(n)]).astype(np.int32)
+        pos[rng.random((n, M)) < 0.05] = -1
+        if trial % 3 == 0:
+            scores = rng.integers(0, 4, size=(n, M)).astype(np.float32) / 8   # heavy ties
+        elif trial % 3 == 1:
+            scores = np.zeros((n, M), np.float32)                             # all tied
+        else:
+            scores = rng.random((n, M)).astype(np.float32)
+        elig = (pos >= 0) & (pos < t0 - R)
+        need = int(min(elig.sum(axis=1).min(), rng.integers(1, M)))
+        if need == 0:
+            continue
+        ev = h2o.select(torch.from_numpy(scores).cuda(), torch.from_numpy(pos).cuda(), t0, R, need)
+        for i in range(n):
+            want = select_evictions(scores[i].astype(np.float64), pos[i], t0, R, need)
+            assert ev[i].cpu().tolist() == want
+
+
+def test_standalone_select_reports_too_few_eligible(h2o):
+    scores = torch.zeros(1, 16, device="cuda")
+    pos = torch.arange(16, dtype=torch.int32, device="cuda")[None]
+    with pytest.raises(h2o.H2OError) as ei:
+        h2o.select(scores, pos, t0=16, R=12, need=5)     # only pos 0..3 are eligible
+    assert ei.value.status == -2
