@@ -1,7 +1,8 @@
 """GPU-vs-oracle comparison for the H2O chunk step (used by the -m gpu tests).
 
 Tolerances (written here, used by every parity test):
-  outputs  float32: |gpu - ref| <= 1e-4 * max(|ref|, 1e-3 * rms(ref)) elementwise
+  outputs  float32: |gpu - ref| <= 1e-4 * max_c |ref[..., c]| (each output row's
+           largest component), elementwise
            bfloat16: |gpu - ref| <= 2e-2 absolute (the relative norm error is also
            reported)
   scores   |gpu - ref| <= 1e-3 * |ref|
@@ -29,8 +30,10 @@ def check_outputs(gpu, ref, dtype, where=""):
     """gpu, ref: float64 arrays of the same shape."""
     err = np.abs(gpu - ref)
     if dtype == torch.float32:
-        rms = float(np.sqrt(np.mean(ref ** 2))) or 1.0
-        bound = OUT_RTOL_F32 * np.maximum(np.abs(ref), 1e-3 * rms)
+        # relative to each output row's magnitude (its largest component): an
+        # elementwise relative bound is undefined where a component crosses zero
+        row = np.abs(ref).max(axis=-1, keepdims=True)
+        bound = OUT_RTOL_F32 * np.maximum(row, 1e-30)
         bad = err > bound
         assert not bad.any(), (f"{where}: {int(bad.sum())} fp32 outputs out of tolerance, "
                                f"max err {err.max():.3e}")
