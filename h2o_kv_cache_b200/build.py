@@ -1,6 +1,6 @@
 """Build libh2o.so in-tree with nvcc for sm_100a.
 
-    python -m h2o_kv_cache_b200.build [--verbose]
+    python h2o_kv_cache_b200/build.py [--verbose]
 
 Each csrc/*.cu is compiled to an object under _build/ (in parallel, skipped when
 the object is newer than its sources) and linked into
