@@ -18,7 +18,7 @@ import torch
 from . import _lib
 from ._lib import (H2O_BF16, H2O_F32, H2O_OK, STATUS_NAMES, lib)
 
-__all__ = ["H2OCache", "H2OError", "select", "lib"]
+__all__ = ["H2OCache", "H2OError", "select", "attend_noalloc", "lib"]
 
 _DTYPES = {torch.float32: H2O_F32, torch.bfloat16: H2O_BF16}
 
@@ -165,3 +165,24 @@ def select(scores, positions, t0: int, R: int, need: int, stream=None):
         _check(lib.h2o_select(_ptr(sc), _ptr(ps), n, M, t0, R, need, _ptr(ev),
                               _stream_ptr(stream, scores.device)))
     return ev
+
+
+def attend_noalloc(q, k, v, k_cache, v_cache, n_valid: int, M: int, out=None, colsum=None,
+                   stream=None):
+    """Attention with summed weights through h2o_attend_noalloc, which allocates
+    no device memory itself (for callers that cannot call cudaMalloc).  Every
+    buffer comes from the caller: q [B,Hq,S,d], k/v [B,Hkv,S,d], k_cache/v_cache
+    [B,Hkv,M,d] (None when n_valid == 0), out [B,Hq,S,d], colsum [B,Hkv,M+S] f32.
+    Returns (out, colsum)."""
+    B, Hq, S, d = q.shape
+    Hkv = k.shape[1]
+    dtype = _DTYPES[q.dtype]
+    if out is None:
+        out = torch.empty_like(q)
+    if colsum is None:
+        colsum = torch.empty(B, Hkv, M + S, dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        _check(lib.h2o_attend_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
+                                      B, Hq, Hkv, d, dtype, M, n_valid, S, _ptr(out), _ptr(colsum),
+                                      _stream_ptr(stream, q.device)))
+    return out, colsum

@@ -2,7 +2,7 @@
 
 Argument marshalling only -- every step of the chunk runs in the library's CUDA
 kernels.  Importing this module loads the in-tree libh2o.so and fails loudly if
-it has not been built (``python -m h2o_kv_cache_b200.build``).
+it has not been built (``python h2o_kv_cache_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -31,12 +31,14 @@ SIGNATURES = {
     "h2o_destroy": (_i32, [_vp]),
     "h2o_last_error": (ctypes.c_char_p, [_vp]),
     "h2o_select": (_i32, [_vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _vp]),
+    "h2o_attend_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i64,
+                                  _i64, _i64, _vp, _vp, _vp]),
 }
 
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
-        raise ImportError(f"{path} is missing: build it with `python -m h2o_kv_cache_b200.build` "
+        raise ImportError(f"{path} is missing: build it with `python h2o_kv_cache_b200/build.py` "
                           "(the library has no fallback path)")
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():

@@ -25,6 +25,11 @@ struct DevBuf {
 
 }  // namespace
 
+int h2o::set_thread_error(int code, const char* msg) {
+  g_thread_err = msg;
+  return code;
+}
+
 struct h2o_ctx {
   int64_t M = 0, R = 0;
   int Hq = 0, Hkv = 0, d = 0, dtype = 0, G = 0, esize = 0;

@@ -64,4 +64,7 @@ cudaError_t launch_scatter(const void* k, const void* v, void* kc, void* vc, flo
                            int32_t* pos, const int32_t* freed, const float* newscore, int BH,
                            int64_t S, int64_t M, int d, int esize, int64_t t0, cudaStream_t st);
 
+// Records msg as this thread's last error (h2o_last_error(NULL)); returns code.
+int set_thread_error(int code, const char* msg);
+
 }  // namespace h2o

@@ -143,6 +143,39 @@ const char* h2o_last_error(h2o_t h);
 int h2o_select(const float* scores, const int32_t* positions, int n_heads, int64_t M,
                int64_t t0, int64_t R, int64_t need, int32_t* evicted, void* stream);
 
+/* Allocation-free attention with summed attention weights.  The paper has no
+ * counterpart to this call: it exists for callers that cannot call cudaMalloc
+ * -- a serving engine that reserves nearly all device memory for its own pool
+ * up front, or latency-critical code that cannot afford cudaMalloc's implicit
+ * device synchronisation.  It allocates nothing: the caller passes every input
+ * and output, and the only scratch (partial column sums and an error word) is
+ * a fixed 16 MiB array in the library's static device memory, which every GPU
+ * that loads the library holds until the process exits.
+ *
+ * Computes steps 1-2 above (attend, summed weights) for one chunk against a
+ * caller-owned cache, without touching any handle state:
+ *   q, out [B, Hq, S, d]; k, v [B, Hkv, S, d]; k_cache, v_cache [B, Hkv, M, d]
+ *   (only slots [0, n_valid) are read; may be NULL when n_valid == 0), all
+ *   device pointers of `dtype`;
+ *   colsum [B, Hkv, M + S] float32 (device): colsum[.., c] for c < M is slot
+ *   c's summed weight (0 for c >= n_valid), colsum[.., M + j] chunk key j's.
+ * Limit: B * Hq * ceil(S / T) * (M + S) <= 4 * 2^20, with T = 128 (bf16, the
+ * tensor-core kernel) or 64 (float32); larger problems return H2O_ESHAPE.
+ * Set-up: the first call on a device looks up the device address of the
+ * scratch array with that device current; make that first call before any
+ * stream capture on the device.
+ * Sharing: every call on a device uses the same scratch, which keeps the last
+ * call's contents; calls whose GPU work overlaps (different streams, or
+ * different host threads, without ordering between them) race on it and give
+ * wrong results.  Order them on one stream or with events.
+ * Errors: H2O_EINVAL (NULL pointer, bad sizes), H2O_ESHAPE (above the limit),
+ * H2O_ECUDA; the message is read with h2o_last_error(NULL).  A bounded
+ * in-kernel wait that runs out is not reported by this call (its outputs are
+ * then invalid); the handle API reports it.                                   */
+int h2o_attend_noalloc(const void* q, const void* k, const void* v, const void* k_cache,
+                       const void* v_cache, int B, int Hq, int Hkv, int d, int dtype, int64_t M,
+                       int64_t n_valid, int64_t S, void* out, float* colsum, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
