@@ -6,27 +6,28 @@
 // also returns the summed attention weights), §1 ¶1 (attention over a
 // fixed-size cache), §1 ¶3 (GQA).
 //
-// One CTA owns 128 query rows of one query head (a row tile) and walks the
-// keys it can see -- the valid cache slots, then the chunk's keys up to its
-// causal limit -- in tiles of 128, twice:
-//   sweep 1  S = Q K^T          (M = 128 queries, N = 128 keys)  -> row max and
-//            sum of exp, i.e. each row's log-sum-exp;
-//   sweep 2  S^T = K Q^T        (M = 128 keys, N = 128 queries), so each
-//            softmax thread owns one key: it forms the exact probabilities
-//            p = exp(s - lse) of its key for the 128 queries, sums them (its
-//            column sum: no cross-thread reduction), and writes them to shared
-//            memory as P^T; then O += P V (M = 128 queries, N = 128 = d) with P
-//            read MN-major.
-// Exact probabilities mean O needs no rescaling.  Each CTA writes one partial
-// row of column sums (per key) that a fixed-order reduction adds up.
+// One CTA owns the same 128 query rows of two query heads A and B that share a
+// KV head (256 rows in all), and walks the keys those rows can see -- the
+// valid cache slots, then the chunk's keys up to the causal limit -- twice:
+//   sweep 1  S_w = Q_w K^T        (per head w: M = 128 queries, N = 256 keys)
+//            -> each row's log-sum-exp;
+//   sweep 2  S^T = K [Q_A; Q_B]^T (M = 128 keys, N = 256 queries): each
+//            softmax thread owns one key, forms its exact probabilities
+//            p = exp(s - lse) for its head's 128 queries, sums them (its column
+//            sum, no cross-thread reduction) and writes them to shared memory
+//            as P^T; then O^T += V^T P^T (M = 128 = d, N = 256 queries), both
+//            operands MN-major.
+// Exact probabilities mean O needs no rescaling.  Every MMA has N = 256: with
+// both operands in shared memory that is what keeps the tensor core near its
+// peak (N = 128 runs at about 70% of it).  Each (head, key) column sum of the
+// CTA goes to one partial row that a fixed-order reduction adds up.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates TMEM
-// and issues the MMAs (one thread), warps 2-9 do the softmax and the epilogue
-// as two warpgroups that share the 128 TMEM lanes (thread = lane) and split
-// each tile's columns in halves -- twice the warps to hide the latency of the
-// exponentials.  TMEM: two 128-column S buffers and a
-// 128-column O accumulator.  Every mbarrier wait is bounded; a wait that runs
-// out sets the kErrTimeout bit of the device error word and all roles exit.
+// Warp roles (320 threads): warp 0 issues TMA loads (one thread), warp 1
+// allocates TMEM and issues the MMAs (one thread), warps 2-5 / 6-9 are the
+// softmax warpgroups of heads A / B (thread = TMEM lane).  TMEM: sweep 1 holds
+// S_A and S_B (256 columns each); sweep 2 holds S^T and O^T (256 each).  Every
+// mbarrier wait is bounded; a wait that runs out sets the kErrTimeout bit of
+// the device error word and all roles exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -41,44 +42,57 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = kUmmaRowTile;   // query rows per CTA
-constexpr int BN = 128;            // keys per tile
+constexpr int BM = kUmmaRowTile;   // query rows per head per CTA
+constexpr int BN = 128;            // keys per TMA tile
 constexpr int D = 128;             // head dimension
-constexpr int NS = 2;              // stages of each of the K and V rings
-constexpr int kThreads = 320;      // TMA warp, MMA warp, two softmax warpgroups
-constexpr uint32_t kAtom = BM * 64 * 2;          // one [128 x 64] bf16 box: 16 KB
+constexpr int kThreads = 320;
+constexpr uint32_t kAtom = 128 * 64 * 2;         // [128 rows x 64 bf16] box: 16 KB
 constexpr uint32_t kTile = 2 * kAtom;            // [128 x 128] bf16: 32 KB
+// shared memory: Q (256 rows, K-major: two 32 KB column atoms), then region R
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTile;               // K ring: NS tiles
-constexpr uint32_t kOffV = kOffK + NS * kTile;          // V ring: NS tiles
-constexpr uint32_t kOffP = kOffV + NS * kTile;
-constexpr uint32_t kOffLse = kOffP + kTile;
-constexpr uint32_t kOffStat = kOffLse + BM * 4;       // row max / sum halves, column-sum hand-over
-constexpr uint32_t kOffBar = kOffStat + 6 * BM * 4;
+constexpr uint32_t kOffR = kOffQ + 2 * kTile;
+// sweep 1: two 64 KB slots, each a 256-key K tile (two 32 KB column atoms)
+constexpr uint32_t kSlot1 = 2 * kTile;
+// sweep 2: three 32 KB slots for K / V tiles, then P^T (128 keys x 256 queries)
+constexpr int NS2 = 3;
+constexpr uint32_t kOffP = kOffR + NS2 * kTile;
+constexpr uint32_t kRBytes = NS2 * kTile + 2 * kTile;   // 160 KB
+constexpr uint32_t kOffLse = kOffR + kRBytes;           // negated base-2 lse, [2][128]
+constexpr uint32_t kOffBar = kOffLse + 2 * BM * 4;
 constexpr int kNumBars = 24;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // slack for 1024-byte alignment
+static_assert(2 * kSlot1 <= kRBytes, "sweep-1 slots fit in R");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;     // 1 s per wait
 
-// barrier indices
-enum { B_Q = 0, B_K_FULL = 1, B_K_EMPTY = B_K_FULL + NS, B_V_FULL = B_K_EMPTY + NS,
-       B_V_EMPTY = B_V_FULL + NS, B_S_FULL = B_V_EMPTY + NS,
-       B_S_EMPTY = B_S_FULL + 2, B_P_FULL = B_S_EMPTY + 2, B_P_EMPTY = B_P_FULL + 1,
-       B_O_FULL = B_P_EMPTY + 1, B_DRAIN = B_O_FULL + 1, B_CS_FULL = B_DRAIN + 1,
-       B_CS_EMPTY = B_CS_FULL + 2 };
-static_assert(B_CS_EMPTY + 1 < kNumBars, "barrier count");
+enum { B_Q = 0, B_R1_FULL = 1, B_R1_EMPTY = 3, B_R2_FULL = 5, B_R2_EMPTY = B_R2_FULL + NS2,
+       B_S_FULL = B_R2_EMPTY + NS2, B_S_EMPTY = B_S_FULL + 2, B_ST_FULL = B_S_EMPTY + 2,
+       B_ST_EMPTY = B_ST_FULL + 1, B_P_FULL = B_ST_EMPTY + 1, B_P_EMPTY = B_P_FULL + 1,
+       B_O_FULL = B_P_EMPTY + 1, B_DRAIN = B_O_FULL + 1 };
+static_assert(B_DRAIN < kNumBars, "barrier count");
 
 struct Params {
   float* partials;
   int* err;
   void* out;
-  int B, Hq, Hkv, G, n_rt;
+  int B, Hq, Hkv, G, n_pg, n_rt;
   int64_t S, M, n_valid;
   float scale_log2;   // (1/sqrt(d)) * log2(e)
 };
+
+// Sweep-2 ring positions: the K / V tiles enter in the order the MMAs use
+// them -- K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1).
+__device__ __forceinline__ int k_pos(int j) { return j == 0 ? 0 : 2 * j - 1; }
+__device__ __forceinline__ int v_pos(int n, int j) { return j + 1 < n ? 2 * j + 2 : 2 * j + 1; }
+
+// Offset of k-step kk (16 columns) inside a K-major tile of `rows` rows whose
+// two 64-column atoms are rows * 128 bytes apart.
+__device__ __forceinline__ uint32_t kmajor_off(int kk, uint32_t rows) {
+  return (uint32_t)(kk >> 2) * rows * 128u + (uint32_t)(kk & 3) * 32u;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -88,34 +102,34 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
-  float* lse2 = reinterpret_cast<float*>(sbase + kOffLse);
+  float* nlse = reinterpret_cast<float*>(sbase + kOffLse);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kOffMisc + 4);
   auto bar = [&](int i) { return base + kOffBar + 8u * (uint32_t)i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work unit: (b, h) major, then row tiles from the last (heaviest) one
-  const int per_bh = p.G * p.n_rt;
+  // ---- work unit: (b, h) major, then row tiles from the last (heaviest), then head pairs
+  const int per_bh = p.n_pg * p.n_rt;
   const int bh = blockIdx.x / per_bh;
   const int k_in = blockIdx.x - bh * per_bh;
-  const int rt = p.n_rt - 1 - k_in / p.G;
-  const int gl = k_in % p.G;
+  const int rt = p.n_rt - 1 - k_in / p.n_pg;
+  const int pg = k_in % p.n_pg;
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
-  const int g = h * p.G + gl;
+  const int gl_a = 2 * pg;                                   // local heads gl_a, gl_a + 1
+  const bool has_b = gl_a + 1 < p.G;
   const int64_t i0 = (int64_t)rt * BM;
-  const int nct = (int)((p.n_valid + BN - 1) / BN);        // cache tiles
-  const int64_t chunk_hi = (i0 + BM < p.S) ? i0 + BM : p.S;  // chunk keys < chunk_hi are visible
+  const int nct = (int)((p.n_valid + BN - 1) / BN);         // cache tiles
+  const int64_t chunk_hi = (i0 + BM < p.S) ? i0 + BM : p.S;   // chunk keys < chunk_hi are visible
   const int nch = (int)((chunk_hi + BN - 1) / BN);
-  const int n = nct + nch;                                   // key tiles per sweep
+  const int n = nct + nch;                                    // 128-key tiles
+  const int n1 = (n + 1) >> 1;                                // sweep-1 256-key tiles
 
   if (threadIdx.x == 0) {
-    // S buffers and P are released / filled by both softmax warpgroups (256
-    // arrivals); the column-sum hand-over by one (128); the rest by one thread
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t cnt = 1;
-      if (i == B_S_EMPTY || i == B_S_EMPTY + 1 || i == B_P_FULL) cnt = 256;
-      if (i >= B_CS_FULL && i < B_CS_EMPTY + 2) cnt = 128;
+      if (i == B_S_EMPTY || i == B_S_EMPTY + 1) cnt = 128;   // one warpgroup
+      if (i == B_ST_EMPTY || i == B_P_FULL) cnt = 256;        // both warpgroups
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -130,6 +144,20 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // tile t (128 keys): tensor map and row offset
+  auto tile_src = [&](int t, bool v, const CUtensorMap*& m, int& y) {
+    if (t < nct) {
+      m = v ? &tm_vc : &tm_kc;
+      y = t * BN;
+    } else if (t < n) {
+      m = v ? &tm_v : &tm_k;
+      y = (t - nct) * BN;
+    } else {  // past the last tile: a box beyond the chunk's rows reads zeros
+      m = v ? &tm_v : &tm_k;
+      y = (int)p.S;
+    }
+  };
+
   if (warp == 0) {
     // =========================================================== TMA producer
     if (lane == 0) {
@@ -138,120 +166,143 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_kc);
       prefetch_tmap(&tm_vc);
-      mbar_arrive_expect_tx(bar(B_Q), kTile);
-      const int zq = b * p.Hq + g;
-      tma_load_3d(base + kOffQ, &tm_q, bar(B_Q), 0, (int)i0, zq);
-      tma_load_3d(base + kOffQ + kAtom, &tm_q, bar(B_Q), 64, (int)i0, zq);
-      // Loads in the order the MMAs consume them.  K ring: sweep 1's tiles, then
-      // sweep 2's; each K stage is freed as soon as its S / S^T MMA is done.  V
-      // ring (sweep 2 only): freed when its PV MMA is done.  Sweep 2 order:
-      // K0, K1, V0, K2, V1, ... so K(j+1) is never queued behind V(j).
-      int k_issued = 0, v_issued = 0;
-      auto load_k = [&](int kit) -> bool {
-        const int stage = kit % NS;
-        if (!mbar_wait(bar(B_K_EMPTY + stage), ((uint32_t)(kit / NS) & 1u) ^ 1u, abort_flag, p.err,
-                       kWaitLimitNs, kErrTimeout))
-          return false;
-        const int t = kit < n ? kit : kit - n;
-        const bool cache = t < nct;
-        const CUtensorMap* mk = cache ? &tm_kc : &tm_k;
-        const int y = cache ? t * BN : (t - nct) * BN;
-        const uint32_t dst = base + kOffK + (uint32_t)stage * kTile;
-        mbar_arrive_expect_tx(bar(B_K_FULL + stage), kTile);
-        tma_load_3d(dst, mk, bar(B_K_FULL + stage), 0, y, bh);
-        tma_load_3d(dst + kAtom, mk, bar(B_K_FULL + stage), 64, y, bh);
-        k_issued = kit + 1;
-        return true;
-      };
-      auto load_v = [&](int j) -> bool {
-        const int stage = j % NS;
-        if (!mbar_wait(bar(B_V_EMPTY + stage), ((uint32_t)(j / NS) & 1u) ^ 1u, abort_flag, p.err,
-                       kWaitLimitNs, kErrTimeout))
-          return false;
-        const bool cache = j < nct;
-        const CUtensorMap* mv = cache ? &tm_vc : &tm_v;
-        const int y = cache ? j * BN : (j - nct) * BN;
-        const uint32_t dst = base + kOffV + (uint32_t)stage * kTile;
-        mbar_arrive_expect_tx(bar(B_V_FULL + stage), kTile);
-        tma_load_3d(dst, mv, bar(B_V_FULL + stage), 0, y, bh);
-        tma_load_3d(dst + kAtom, mv, bar(B_V_FULL + stage), 64, y, bh);
-        v_issued = j + 1;
-        return true;
-      };
+      // Q: rows of head A then head B, each split into two 64-column atoms
+      const int zq = b * p.Hq + h * p.G + gl_a;
+      mbar_arrive_expect_tx(bar(B_Q), 2 * kTile);
+      for (int hw = 0; hw < 2; ++hw)
+        for (int at = 0; at < 2; ++at)
+          tma_load_3d(base + kOffQ + at * 2 * kAtom + hw * kAtom, &tm_q, bar(B_Q), at * 64, (int)i0,
+                      zq + hw);
       bool ok = true;
-      for (int kit = 0; ok && kit <= n; ++kit) ok = load_k(kit);      // sweep 1, then K0 of sweep 2
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 1 < n) ok = load_k(n + j + 1);
-        if (ok) ok = load_v(j);
+      // sweep 1: 256-key K tiles into two 64 KB slots
+      for (int u = 0; ok && u < n1; ++u) {
+        const int s = u & 1;
+        ok = mbar_wait(bar(B_R1_EMPTY + s), ((uint32_t)(u >> 1) & 1u) ^ 1u, abort_flag, p.err,
+                       kWaitLimitNs, kErrTimeout);
+        if (!ok) break;
+        const uint32_t dst = base + kOffR + (uint32_t)s * kSlot1;
+        mbar_arrive_expect_tx(bar(B_R1_FULL + s), kSlot1);
+        for (int half = 0; half < 2; ++half) {
+          const CUtensorMap* m;
+          int y;
+          tile_src(2 * u + half, false, m, y);
+          for (int at = 0; at < 2; ++at)
+            tma_load_3d(dst + at * 2 * kAtom + half * kAtom, m, bar(B_R1_FULL + s), at * 64, y, bh);
+        }
       }
-      // drain: the last loads of each ring have landed before the CTA may exit
-      for (int it = k_issued - NS < 0 ? 0 : k_issued - NS; it < k_issued; ++it)
-        mbar_wait(bar(B_K_FULL + it % NS), (uint32_t)(it / NS) & 1u, abort_flag, p.err,
-                  kWaitLimitNs, kErrTimeout);
-      for (int it = v_issued - NS < 0 ? 0 : v_issued - NS; it < v_issued; ++it)
-        mbar_wait(bar(B_V_FULL + it % NS), (uint32_t)(it / NS) & 1u, abort_flag, p.err,
+      // sweep 2 reuses R: wait until every sweep-1 slot has been read
+      for (int s = 0; ok && s < 2; ++s) {
+        const int fills = (n1 - s + 1) >> 1;
+        if (fills > 0)
+          ok = mbar_wait(bar(B_R1_EMPTY + s), (uint32_t)(fills - 1) & 1u, abort_flag, p.err,
+                         kWaitLimitNs, kErrTimeout);
+      }
+      int issued = 0;
+      for (int pos = 0; ok && pos < 2 * n; ++pos) {
+        const int slot = pos % NS2;
+        ok = mbar_wait(bar(B_R2_EMPTY + slot), ((uint32_t)(pos / NS2) & 1u) ^ 1u, abort_flag, p.err,
+                       kWaitLimitNs, kErrTimeout);
+        if (!ok) break;
+        bool is_v;
+        int t;
+        if (pos == 0) { is_v = false; t = 0; }
+        else if (pos == 2 * n - 1) { is_v = true; t = n - 1; }
+        else if (pos & 1) { is_v = false; t = (pos + 1) >> 1; }
+        else { is_v = true; t = (pos >> 1) - 1; }
+        const CUtensorMap* m;
+        int y;
+        tile_src(t, is_v, m, y);
+        const uint32_t dst = base + kOffR + (uint32_t)slot * kTile;
+        mbar_arrive_expect_tx(bar(B_R2_FULL + slot), kTile);
+        tma_load_3d(dst, m, bar(B_R2_FULL + slot), 0, y, bh);
+        tma_load_3d(dst + kAtom, m, bar(B_R2_FULL + slot), 64, y, bh);
+        issued = pos + 1;
+      }
+      // drain: the last load of each slot has landed before the CTA may exit
+      for (int pos = issued - NS2 < 0 ? 0 : issued - NS2; pos < issued; ++pos)
+        mbar_wait(bar(B_R2_FULL + pos % NS2), (uint32_t)(pos / NS2) & 1u, abort_flag, p.err,
                   kWaitLimitNs, kErrTimeout);
     }
   } else if (warp == 1) {
     // =========================================================== MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);
-      const uint32_t idesc_pv = idesc_bf16(128, 128, 1, 1);
+      const uint32_t idesc_kk = idesc_bf16(128, 256, 0, 0);   // both operands K-major
+      const uint32_t idesc_mn = idesc_bf16(128, 256, 1, 1);   // both operands MN-major
       const uint32_t q_addr = base + kOffQ;
       const uint32_t p_addr = base + kOffP;
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag, p.err, kWaitLimitNs, kErrTimeout);
-      // issues S (sweep 1: Q K^T) or S^T (sweep 2: K Q^T) for iteration it
-      auto issue_s = [&](int it) -> bool {
-        const int stage = it % NS;
-        const int sb = it & 1;
-        if (!mbar_wait(bar(B_K_FULL + stage), (uint32_t)(it / NS) & 1u, abort_flag, p.err,
-                       kWaitLimitNs, kErrTimeout))
-          return false;
-        if (!mbar_wait(bar(B_S_EMPTY + sb), ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, p.err,
-                       kWaitLimitNs, kErrTimeout))
-          return false;
+      // ---- sweep 1
+      for (int u = 0; ok && u < n1; ++u) {
+        const int s = u & 1;
+        ok = mbar_wait(bar(B_R1_FULL + s), (uint32_t)(u >> 1) & 1u, abort_flag, p.err, kWaitLimitNs,
+                       kErrTimeout);
+        const uint32_t k_addr = base + kOffR + (uint32_t)s * kSlot1;
+        for (int w = 0; ok && w < 2; ++w) {
+          ok = mbar_wait(bar(B_S_EMPTY + w), ((uint32_t)u & 1u) ^ 1u, abort_flag, p.err, kWaitLimitNs,
+                         kErrTimeout);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t da = smem_desc_sw128(q_addr + (uint32_t)w * kAtom + kmajor_off(kk, 256), 16, 1024);
+            const uint64_t db = smem_desc_sw128(k_addr + kmajor_off(kk, 256), 16, 1024);
+            umma_bf16(tmem + (uint32_t)w * 256u, da, db, idesc_kk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar(B_S_FULL + w));
+        }
+        if (ok) umma_commit(bar(B_R1_EMPTY + s));
+      }
+      // ---- sweep 2: S^T(0), S^T(1), O^T(0), S^T(2), O^T(1), ...
+      auto issue_st = [&](int j) -> bool {
+        // TMEM columns 0-255: head A's last sweep-1 S, then S^T(j - 1), must have been read
+        bool w_ok = (j == 0)
+            ? mbar_wait(bar(B_S_EMPTY + 0), ((uint32_t)n1 & 1u) ^ 1u, abort_flag, p.err, kWaitLimitNs, kErrTimeout)
+            : mbar_wait(bar(B_ST_EMPTY), (uint32_t)(j - 1) & 1u, abort_flag, p.err, kWaitLimitNs, kErrTimeout);
+        const int pos = k_pos(j), slot = pos % NS2;
+        if (w_ok)
+          w_ok = mbar_wait(bar(B_R2_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, p.err,
+                           kWaitLimitNs, kErrTimeout);
+        if (!w_ok) return false;
         tc_fence_after();
-        const uint32_t k_addr = base + kOffK + (uint32_t)stage * kTile;
-        const uint32_t d_tmem = tmem + (uint32_t)sb * 128u;
+        const uint32_t k_addr = base + kOffR + (uint32_t)slot * kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)(kk >> 2) * kAtom + (uint32_t)(kk & 3) * 32u;
-          const uint64_t dq = smem_desc_sw128(q_addr + off, 16, 1024);
-          const uint64_t dk = smem_desc_sw128(k_addr + off, 16, 1024);
-          if (it < n) umma_bf16(d_tmem, dq, dk, idesc_s, kk > 0 ? 1u : 0u);
-          else umma_bf16(d_tmem, dk, dq, idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t da = smem_desc_sw128(k_addr + kmajor_off(kk, 128), 16, 1024);
+          const uint64_t db = smem_desc_sw128(q_addr + kmajor_off(kk, 256), 16, 1024);
+          umma_bf16(tmem, da, db, idesc_kk, kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar(B_S_FULL + sb));
-        umma_commit(bar(B_K_EMPTY + stage));
+        umma_commit(bar(B_ST_FULL));
+        umma_commit(bar(B_R2_EMPTY + slot));
         return true;
       };
-      for (int it = 0; ok && it < n; ++it) ok = issue_s(it);
-      if (ok) ok = issue_s(n);
-      for (int j = 0; ok && j < n; ++j) {
-        const int it = n + j;
-        if (j + 1 < n) ok = issue_s(it + 1);
-        if (!ok) break;
-        if (!mbar_wait(bar(B_P_FULL), (uint32_t)j & 1u, abort_flag, p.err, kWaitLimitNs, kErrTimeout)) {
-          ok = false;
-          break;
-        }
-        const int stage = j % NS;
-        if (!mbar_wait(bar(B_V_FULL + stage), (uint32_t)(j / NS) & 1u, abort_flag, p.err,
-                       kWaitLimitNs, kErrTimeout)) {
-          ok = false;
-          break;
-        }
+      auto issue_ot = [&](int j) -> bool {
+        bool w_ok = mbar_wait(bar(B_P_FULL), (uint32_t)j & 1u, abort_flag, p.err, kWaitLimitNs, kErrTimeout);
+        // TMEM columns 256-511: head B's last sweep-1 S must have been read
+        if (w_ok && j == 0)
+          w_ok = mbar_wait(bar(B_S_EMPTY + 1), ((uint32_t)n1 & 1u) ^ 1u, abort_flag, p.err,
+                           kWaitLimitNs, kErrTimeout);
+        const int pos = v_pos(n, j), slot = pos % NS2;
+        if (w_ok)
+          w_ok = mbar_wait(bar(B_R2_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, p.err,
+                           kWaitLimitNs, kErrTimeout);
+        if (!w_ok) return false;
         tc_fence_after();
-        const uint32_t v_addr = base + kOffV + (uint32_t)stage * kTile;
+        const uint32_t v_addr = base + kOffR + (uint32_t)slot * kTile;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t dp = smem_desc_sw128(p_addr + (uint32_t)kk * 2048u, kAtom, 1024);
-          const uint64_t dv = smem_desc_sw128(v_addr + (uint32_t)kk * 2048u, kAtom, 1024);
-          umma_bf16(tmem + kColO, dp, dv, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t da = smem_desc_sw128(v_addr + (uint32_t)kk * 2048u, kAtom, 1024);
+          const uint64_t db = smem_desc_sw128(p_addr + (uint32_t)kk * 2048u, kAtom, 1024);
+          umma_bf16(tmem + 256u, da, db, idesc_mn, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar(B_P_EMPTY));
-        umma_commit(bar(B_V_EMPTY + stage));
+        umma_commit(bar(B_R2_EMPTY + slot));
+        return true;
+      };
+      for (int j = 0; ok && j < n; ++j) {
+        ok = issue_st(j);
+        if (ok && j > 0) ok = issue_ot(j - 1);
       }
+      if (ok) ok = issue_ot(n - 1);
       umma_commit(bar(B_O_FULL));
       // every MMA issued has completed before TMEM is released
       umma_commit(bar(B_DRAIN));
@@ -259,187 +310,164 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else {
     // =========================================================== softmax / epilogue
-    // Two warpgroups share every TMEM lane: warpgroup hc (0: warps 2-5, 1: warps
-    // 6-9) takes columns [64 hc, 64 hc + 64) of each S / S^T / O tile.
-    const int hc = (warp - 2) >> 2;
+    const int w = (warp - 2) >> 2;                    // 0: head A, 1: head B
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                 // TMEM lane owned by this thread
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)hc * 64u;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const int64_t S = p.S, M = p.M, nv = p.n_valid;
     const float c = p.scale_log2;
-    float* sm_m = reinterpret_cast<float*>(sbase + kOffStat);        // [2][128]
-    float* sm_l = sm_m + 2 * BM;                                      // [2][128]
-    float* cs_buf = sm_l + 2 * BM;                                    // [2][128]
+    const bool head_ok = w == 0 || has_b;
     bool ok = true;
 
-    // ----- sweep 1: thread = query row i0 + r, keys of its column half
+    // ----- sweep 1: thread = query row i0 + r of head w; running (max, sum).
+    // The sum is kept against a reference max that is only raised when a
+    // 64-key chunk's max exceeds it by more than 8 (log2 units), so the
+    // exponentials of a chunk never wait for that chunk's max.
     const int64_t row_i = i0 + r;
+    const int64_t row_lim = (row_i + 1 < S) ? row_i + 1 : S;   // chunk keys < row_lim are seen
     float m = -INFINITY, l = 0.f;
-    for (int it = 0; ok && it < n; ++it) {
-      const int sb = it & 1;
-      // tcgen05.ld is warp-collective: the whole warp proceeds or stops together
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + sb), (uint32_t)(it >> 1) & 1u,
-                                             abort_flag, p.err, kWaitLimitNs, kErrTimeout));
+    const uint32_t s_tmem = lane_base + (uint32_t)w * 256u;
+    for (int u = 0; ok && u < n1; ++u) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + w), (uint32_t)u & 1u, abort_flag, p.err,
+                                             kWaitLimitNs, kErrTimeout));
       if (!ok) break;
       tc_fence_after();
-      uint32_t v[2][32];
-      tmem_ld32(lane_base + (uint32_t)sb * 128u, v[0]);
-      tmem_ld32(lane_base + (uint32_t)sb * 128u + 32u, v[1]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_S_EMPTY + sb));
-      const bool cache = it < nct;
-      const int64_t key0 = (cache ? (int64_t)it * BN : (int64_t)(it - nct) * BN) + hc * 64;
-      // keys visible to this row: cache slots < n_valid; chunk keys <= row_i (and < S)
-      const int64_t lim = cache ? nv : ((row_i + 1 < S) ? row_i + 1 : S);
-      const int nvis = (int)(lim - key0 > 64 ? 64 : (lim - key0 < 0 ? 0 : lim - key0));
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (nvis == 64) {
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          const float x = __uint_as_float(v[k >> 5][k & 31]) * c;
-          v[k >> 5][k & 31] = __float_as_uint(x);
-          mx4[k & 3] = fmaxf(mx4[k & 3], x);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {                 // 64 keys per chunk
+        uint32_t v[2][32];
+        tmem_ld32(s_tmem + ch * 64, v[0]);
+        tmem_ld32(s_tmem + ch * 64 + 32, v[1]);
+        tmem_wait_ld();
+        if (ch == 3) {
+          tc_fence_before();
+          mbar_arrive(bar(B_S_EMPTY + w));
         }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          const float x = k < nvis ? __uint_as_float(v[k >> 5][k & 31]) * c : -INFINITY;
-          v[k >> 5][k & 31] = __float_as_uint(x);
-          mx4[k & 3] = fmaxf(mx4[k & 3], x);
+        const int t = 2 * u + (ch >> 1);
+        int nvis = 0;
+        if (t < n) {
+          const bool cache = t < nct;
+          const int64_t key0 = (cache ? (int64_t)t * BN : (int64_t)(t - nct) * BN) + (ch & 1) * 64;
+          const int64_t lim = cache ? nv : row_lim;
+          nvis = (int)(lim - key0 > 64 ? 64 : (lim - key0 < 0 ? 0 : lim - key0));
         }
-      }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      if (mx > -INFINITY) {
-        const float mn = fmaxf(m, mx);
+        if (nvis < 64) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k)
+            if (k >= nvis) v[k >> 5][k & 31] = __float_as_uint(-INFINITY);
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float nm = -m;
 #pragma unroll
-        for (int k = 0; k < 64; ++k) s8[k & 7] += ex2(__uint_as_float(v[k >> 5][k & 31]) - mn);
-        const float sum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-        l = (m == -INFINITY ? 0.f : l * ex2(m - mn)) + sum;
-        m = mn;
+        for (int k = 0; k < 64; ++k) {
+          const float x = __uint_as_float(v[k >> 5][k & 31]);
+          mx4[k & 3] = fmaxf(mx4[k & 3], x);
+          s8[k & 7] += ex2(fmaf(x, c, nm));
+        }
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c;
+        if (mx > m + 8.f) {
+          // rare: raise the reference and recompute this chunk's sum against it
+#pragma unroll
+          for (int k = 0; k < 8; ++k) s8[k] = 0.f;
+#pragma unroll
+          for (int k = 0; k < 64; ++k) s8[k & 7] += ex2(fmaf(__uint_as_float(v[k >> 5][k & 31]), c, -mx));
+          l = (m == -INFINITY) ? 0.f : l * ex2(m - mx);
+          m = mx;
+        }
+        l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+        __syncwarp();
       }
-      __syncwarp();
     }
-    // combine the two column halves of each row into its log-sum-exp (base 2)
-    sm_m[hc * BM + r] = m;
-    sm_l[hc * BM + r] = l;
-    named_bar_sync(1, 256);
-    if (hc == 0) {
-      const float ma = sm_m[r], mb = sm_m[BM + r];
-      const float la = sm_l[r], lb = sm_l[BM + r];
-      const float mm = fmaxf(ma, mb);
-      const float ll = (ma == -INFINITY ? 0.f : la * ex2(ma - mm)) + (mb == -INFINITY ? 0.f : lb * ex2(mb - mm));
-      // stored negated: sweep 2 forms s * c - lse with one FFMA; -inf zeroes invalid rows
-      lse2[r] = (row_i < S && ll > 0.f) ? -(mm + lg2(ll)) : -INFINITY;
-    }
-    named_bar_sync(1, 256);
-    float nl[64];
-#pragma unroll
-    for (int k = 0; k < 64; k += 4) {
-      const float4 t4 = *reinterpret_cast<const float4*>(lse2 + hc * 64 + k);
-      nl[k] = t4.x; nl[k + 1] = t4.y; nl[k + 2] = t4.z; nl[k + 3] = t4.w;
-    }
+    // negated base-2 log-sum-exp of each row; -inf zeroes rows past S and a missing head B
+    nlse[w * BM + r] = (head_ok && row_i < S && l > 0.f) ? -(m + lg2(l)) : -INFINITY;
+    named_bar_sync(1 + w, 128);
 
-    // ----- sweep 2: thread = key (lane r of the S^T tile), query columns of its half
-    float* part = p.partials + ((int64_t)bh * (p.G * p.n_rt) + (gl * p.n_rt + rt)) * (M + S);
-    const uint32_t p_row = base + kOffP + (uint32_t)hc * kAtom + (uint32_t)(r >> 3) * 1024u +
+    // ----- sweep 2: thread = key (lane r of S^T), the 128 query columns of head w
+    float* part = p.partials + ((int64_t)bh * (p.G * p.n_rt) + ((gl_a + w) * p.n_rt + rt)) * (M + S);
+    const uint32_t p_row = base + kOffP + (uint32_t)(2 * w) * kAtom + (uint32_t)(r >> 3) * 1024u +
                            (uint32_t)(r & 7) * 128u;
+    const float* nl_w = nlse + w * BM;
+    const uint32_t st_tmem = lane_base + (uint32_t)w * 128u;
     for (int j = 0; ok && j < n; ++j) {
-      const int it = n + j;
-      const int sb = it & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + sb), (uint32_t)(it >> 1) & 1u,
-                                             abort_flag, p.err, kWaitLimitNs, kErrTimeout));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ST_FULL), (uint32_t)j & 1u, abort_flag, p.err,
+                                             kWaitLimitNs, kErrTimeout));
       if (!ok) break;
       tc_fence_after();
-      uint32_t v[2][32];
-      tmem_ld32(lane_base + (uint32_t)sb * 128u, v[0]);
-      tmem_ld32(lane_base + (uint32_t)sb * 128u + 32u, v[1]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_S_EMPTY + sb));
       const bool cache = j < nct;
       const int64_t key = cache ? (int64_t)j * BN + r : (int64_t)(j - nct) * BN + r;
       const bool key_ok = cache ? key < nv : key < S;
       // chunk key `key` is seen by query columns q with i0 + q >= key
-      const int qmin = (cache ? 0 : (int)(key - i0 > 0 ? key - i0 : 0)) - hc * 64;
+      const int qmin = cache ? 0 : (int)(key - i0 > 0 ? key - i0 : 0);
+      const bool full = key_ok && qmin == 0;
       float cs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
-      if (key_ok && qmin <= 0) {
+      uint32_t pk[64];
 #pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          const float e0 = ex2(fmaf(__uint_as_float(v[k >> 5][k & 31]), c, nl[k]));
-          const float e1 = ex2(fmaf(__uint_as_float(v[k >> 5][(k + 1) & 31]), c, nl[k + 1]));
-          cs8[k & 7] += e0;
-          cs8[(k + 1) & 7] += e1;
-          pk[k >> 1] = pack_bf16(e0, e1);
+      for (int hf = 0; hf < 2; ++hf) {                 // 64 queries at a time
+        uint32_t v[2][32];
+        tmem_ld32(st_tmem + hf * 64, v[0]);
+        tmem_ld32(st_tmem + hf * 64 + 32, v[1]);
+        tmem_wait_ld();
+        if (hf == 1) {
+          tc_fence_before();
+          mbar_arrive(bar(B_ST_EMPTY));
         }
-      } else {
 #pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          float e0 = ex2(fmaf(__uint_as_float(v[k >> 5][k & 31]), c, nl[k]));
-          float e1 = ex2(fmaf(__uint_as_float(v[k >> 5][(k + 1) & 31]), c, nl[k + 1]));
-          e0 = (key_ok && k >= qmin) ? e0 : 0.f;
-          e1 = (key_ok && k + 1 >= qmin) ? e1 : 0.f;
-          cs8[k & 7] += e0;
-          cs8[(k + 1) & 7] += e1;
-          pk[k >> 1] = pack_bf16(e0, e1);
+        for (int k = 0; k < 64; k += 4) {
+          const float4 n4 = *reinterpret_cast<const float4*>(nl_w + hf * 64 + k);
+          const float nlk[4] = {n4.x, n4.y, n4.z, n4.w};
+          float e[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            e[i] = ex2(fmaf(__uint_as_float(v[(k + i) >> 5][(k + i) & 31]), c, nlk[i]));
+            if (!full) e[i] = (key_ok && hf * 64 + k + i >= qmin) ? e[i] : 0.f;
+            cs8[(k + i) & 7] += e[i];
+          }
+          pk[hf * 32 + (k >> 1)] = pack_bf16(e[0], e[1]);
+          pk[hf * 32 + (k >> 1) + 1] = pack_bf16(e[2], e[3]);
         }
       }
-      float cs = ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
+      const float cs = ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
+      if (key_ok && head_ok) part[cache ? key : M + key] = cs;
+      // P^T row r -> query blocks 2w, 2w + 1, once the previous O^T MMA is done
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
                                              p.err, kWaitLimitNs, kErrTimeout));
       if (!ok) break;
-      // P^T row r (key) -> MN-major P tile, query block hc, 16-byte chunks
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const uint32_t addr = p_row + (((uint32_t)c8 ^ (uint32_t)(r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[c8 * 4]),
-                     "r"(pk[c8 * 4 + 1]), "r"(pk[c8 * 4 + 2]), "r"(pk[c8 * 4 + 3])
+      for (int ch = 0; ch < 16; ++ch) {
+        const uint32_t addr = p_row + (uint32_t)(ch >> 3) * kAtom +
+                              ((((uint32_t)ch & 7u) ^ (uint32_t)(r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[ch * 4]),
+                     "r"(pk[ch * 4 + 1]), "r"(pk[ch * 4 + 2]), "r"(pk[ch * 4 + 3])
                      : "memory");
       }
       fence_async_smem();
       mbar_arrive(bar(B_P_FULL));
-      // the key's column sum over all 128 queries: warpgroup 1 hands its half over
-      const int cb = j & 1;
-      const uint32_t cph = (uint32_t)(j >> 1) & 1u;
-      if (hc == 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_EMPTY + cb), cph ^ 1u, abort_flag, p.err,
-                                               kWaitLimitNs, kErrTimeout));
-        if (!ok) break;
-        cs_buf[cb * BM + r] = cs;
-        mbar_arrive(bar(B_CS_FULL + cb));
-      } else {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_FULL + cb), cph, abort_flag, p.err,
-                                               kWaitLimitNs, kErrTimeout));
-        if (!ok) break;
-        cs += cs_buf[cb * BM + r];
-        mbar_arrive(bar(B_CS_EMPTY + cb));
-        if (key_ok) part[cache ? key : M + key] = cs;
-      }
     }
 
-    // ----- epilogue: thread = query row i0 + r, output columns of its half
+    // ----- epilogue: O^T (lane = d, columns = queries) -> out rows via shared memory
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), 0, abort_flag, p.err,
                                                    kWaitLimitNs, kErrTimeout));
     if (ok) {
       tc_fence_after();
-      uint32_t o[2][32];
-      tmem_ld32(lane_base + kColO, o[0]);
-      tmem_ld32(lane_base + kColO + 32u, o[1]);
-      tmem_wait_ld();
-      if (p.out != nullptr && row_i < S) {
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
-                              (((int64_t)b * p.Hq + g) * S + row_i) * D + hc * 64;
+      // every MMA has completed: R is free; head w's [128 queries x 128 d] goes to R + w * 32 KB
+      __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sbase + kOffR + (uint32_t)w * kTile);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + 256u + (uint32_t)w * 128u + ch * 32, o);
+        tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 64; k += 8) {
-          uint4 w;
-          w.x = pack_bf16(__uint_as_float(o[k >> 5][k & 31]), __uint_as_float(o[k >> 5][(k + 1) & 31]));
-          w.y = pack_bf16(__uint_as_float(o[k >> 5][(k + 2) & 31]), __uint_as_float(o[k >> 5][(k + 3) & 31]));
-          w.z = pack_bf16(__uint_as_float(o[k >> 5][(k + 4) & 31]), __uint_as_float(o[k >> 5][(k + 5) & 31]));
-          w.w = pack_bf16(__uint_as_float(o[k >> 5][(k + 6) & 31]), __uint_as_float(o[k >> 5][(k + 7) & 31]));
-          *reinterpret_cast<uint4*>(orow + k) = w;
-        }
+        for (int k = 0; k < 32; ++k) stage[(ch * 32 + k) * D + r] = __float2bfloat16_rn(__uint_as_float(o[k]));
+      }
+      named_bar_sync(1 + w, 128);
+      const int64_t qi = i0 + r;                       // thread r copies query row r
+      if (p.out != nullptr && head_ok && qi < S) {
+        const int g = h * p.G + gl_a + w;
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                              (((int64_t)b * p.Hq + g) * S + qi) * D);
+        const uint4* src = reinterpret_cast<const uint4*>(stage + r * D);
+#pragma unroll
+        for (int k = 0; k < D * 2 / 16; ++k) dst[k] = src[k];
       }
     }
   }
@@ -505,6 +533,7 @@ cudaError_t launch_attn_umma(const AttnArgs& a, cudaStream_t st) {
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.G = a.Hq / a.Hkv;
+  p.n_pg = (p.G + 1) / 2;
   p.n_rt = (int)((a.S + BM - 1) / BM);
   p.S = a.S;
   p.M = a.M;
@@ -512,7 +541,7 @@ cudaError_t launch_attn_umma(const AttnArgs& a, cudaStream_t st) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   e = cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int64_t grid = BHkv * p.G * p.n_rt;
+  const int64_t grid = BHkv * p.n_pg * p.n_rt;
   attn_umma_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, mkc, mvc, p);
   return cudaGetLastError();
 }
