@@ -94,6 +94,68 @@ __device__ __forceinline__ uint32_t kmajor_off(int kk, uint32_t rows) {
   return (uint32_t)(kk >> 2) * rows * 128u + (uint32_t)(kk & 3) * 32u;
 }
 
+// Sweep 1: one 64-key chunk of a row (x = raw scores in v, nvis of them
+// visible) folded into the running (m, l), base 2.
+__device__ __forceinline__ void row_chunk(uint32_t (&v)[2][32], int nvis, float c, float& m, float& l) {
+  if (nvis < 64) {
+#pragma unroll
+    for (int k = 0; k < 64; ++k)
+      if (k >= nvis) v[k >> 5][k & 31] = __float_as_uint(-INFINITY);
+  }
+  float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const float nm = -m;
+#pragma unroll
+  for (int k = 0; k < 64; ++k) {
+    const float x = __uint_as_float(v[k >> 5][k & 31]);
+    mx4[k & 3] = fmaxf(mx4[k & 3], x);
+    s8[k & 7] += ex2(fmaf(x, c, nm));
+  }
+  const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c;
+  if (mx > m + 8.f) {
+    // rare: raise the reference and recompute this chunk's sum against it
+#pragma unroll
+    for (int k = 0; k < 8; ++k) s8[k] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 64; ++k) s8[k & 7] += ex2(fmaf(__uint_as_float(v[k >> 5][k & 31]), c, -mx));
+    l = (m == -INFINITY) ? 0.f : l * ex2(m - mx);
+    m = mx;
+  }
+  l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+}
+
+// Sweep 2: 64 query columns of a key's S^T row -> p = 2^(s c - lse) (zero where
+// masked), column-sum terms into cs8, packed bf16 pairs into pk.
+template <bool kFull>
+__device__ __forceinline__ void key_half(const uint32_t (&v)[2][32], const float* nl, float c,
+                                         bool key_ok, int qmin, float (&cs8)[8], uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int k = 0; k < 64; k += 4) {
+    const float4 n4 = *reinterpret_cast<const float4*>(nl + k);
+    const float nlk[4] = {n4.x, n4.y, n4.z, n4.w};
+    float e[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      e[i] = ex2(fmaf(__uint_as_float(v[(k + i) >> 5][(k + i) & 31]), c, nlk[i]));
+      if (!kFull) e[i] = (key_ok && k + i >= qmin) ? e[i] : 0.f;
+      cs8[(k + i) & 7] += e[i];
+    }
+    pk[k >> 1] = pack_bf16(e[0], e[1]);
+    pk[(k >> 1) + 1] = pack_bf16(e[2], e[3]);
+  }
+}
+
+// Sweep 2: a key's 64-query half of P^T (packed) into its 128-byte swizzled row.
+__device__ __forceinline__ void store_p_half(uint32_t row_addr, int r, const uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int c8 = 0; c8 < 8; ++c8) {
+    const uint32_t addr = row_addr + ((((uint32_t)c8) ^ (uint32_t)(r & 7)) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[c8 * 4]),
+                 "r"(pk[c8 * 4 + 1]), "r"(pk[c8 * 4 + 2]), "r"(pk[c8 * 4 + 3])
+                 : "memory");
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
@@ -327,13 +389,28 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int64_t row_lim = (row_i + 1 < S) ? row_i + 1 : S;   // chunk keys < row_lim are seen
     float m = -INFINITY, l = 0.f;
     const uint32_t s_tmem = lane_base + (uint32_t)w * 256u;
+    auto nvis_of = [&](int t, int half64) -> int {
+      if (t >= n) return 0;
+      const bool cache = t < nct;
+      const int64_t key0 = (cache ? (int64_t)t * BN : (int64_t)(t - nct) * BN) + half64 * 64;
+      const int64_t lim = cache ? nv : row_lim;
+      return (int)(lim - key0 > 64 ? 64 : (lim - key0 < 0 ? 0 : lim - key0));
+    };
     for (int u = 0; ok && u < n1; ++u) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + w), (uint32_t)u & 1u, abort_flag, p.err,
                                              kWaitLimitNs, kErrTimeout));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {                 // 64 keys per chunk
+      for (int ch = 0; ch < 2; ++ch) {                 // keys 0-127 of the tile, 64 at a time
+        uint32_t v[2][32];
+        tmem_ld32(s_tmem + ch * 64, v[0]);
+        tmem_ld32(s_tmem + ch * 64 + 32, v[1]);
+        tmem_wait_ld();
+        row_chunk(v, nvis_of(2 * u, ch), c, m, l);
+      }
+#pragma unroll 1
+      for (int ch = 2; ch < 4; ++ch) {
         uint32_t v[2][32];
         tmem_ld32(s_tmem + ch * 64, v[0]);
         tmem_ld32(s_tmem + ch * 64 + 32, v[1]);
@@ -342,41 +419,9 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tc_fence_before();
           mbar_arrive(bar(B_S_EMPTY + w));
         }
-        const int t = 2 * u + (ch >> 1);
-        int nvis = 0;
-        if (t < n) {
-          const bool cache = t < nct;
-          const int64_t key0 = (cache ? (int64_t)t * BN : (int64_t)(t - nct) * BN) + (ch & 1) * 64;
-          const int64_t lim = cache ? nv : row_lim;
-          nvis = (int)(lim - key0 > 64 ? 64 : (lim - key0 < 0 ? 0 : lim - key0));
-        }
-        if (nvis < 64) {
-#pragma unroll
-          for (int k = 0; k < 64; ++k)
-            if (k >= nvis) v[k >> 5][k & 31] = __float_as_uint(-INFINITY);
-        }
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const float nm = -m;
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          const float x = __uint_as_float(v[k >> 5][k & 31]);
-          mx4[k & 3] = fmaxf(mx4[k & 3], x);
-          s8[k & 7] += ex2(fmaf(x, c, nm));
-        }
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c;
-        if (mx > m + 8.f) {
-          // rare: raise the reference and recompute this chunk's sum against it
-#pragma unroll
-          for (int k = 0; k < 8; ++k) s8[k] = 0.f;
-#pragma unroll
-          for (int k = 0; k < 64; ++k) s8[k & 7] += ex2(fmaf(__uint_as_float(v[k >> 5][k & 31]), c, -mx));
-          l = (m == -INFINITY) ? 0.f : l * ex2(m - mx);
-          m = mx;
-        }
-        l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-        __syncwarp();
+        row_chunk(v, nvis_of(2 * u + 1, ch - 2), c, m, l);
       }
+      __syncwarp();
     }
     // negated base-2 log-sum-exp of each row; -inf zeroes rows past S and a missing head B
     nlse[w * BM + r] = (head_ok && row_i < S && l > 0.f) ? -(m + lg2(l)) : -INFINITY;
@@ -398,50 +443,38 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const bool key_ok = cache ? key < nv : key < S;
       // chunk key `key` is seen by query columns q with i0 + q >= key
       const int qmin = cache ? 0 : (int)(key - i0 > 0 ? key - i0 : 0);
-      const bool full = key_ok && qmin == 0;
+      const bool full = __all_sync(0xffffffffu, key_ok && qmin == 0);
       float cs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[64];
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {                 // 64 queries at a time
+      uint32_t pk[32];
+      {
         uint32_t v[2][32];
-        tmem_ld32(st_tmem + hf * 64, v[0]);
-        tmem_ld32(st_tmem + hf * 64 + 32, v[1]);
+        tmem_ld32(st_tmem, v[0]);
+        tmem_ld32(st_tmem + 32, v[1]);
         tmem_wait_ld();
-        if (hf == 1) {
-          tc_fence_before();
-          mbar_arrive(bar(B_ST_EMPTY));
-        }
-#pragma unroll
-        for (int k = 0; k < 64; k += 4) {
-          const float4 n4 = *reinterpret_cast<const float4*>(nl_w + hf * 64 + k);
-          const float nlk[4] = {n4.x, n4.y, n4.z, n4.w};
-          float e[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            e[i] = ex2(fmaf(__uint_as_float(v[(k + i) >> 5][(k + i) & 31]), c, nlk[i]));
-            if (!full) e[i] = (key_ok && hf * 64 + k + i >= qmin) ? e[i] : 0.f;
-            cs8[(k + i) & 7] += e[i];
-          }
-          pk[hf * 32 + (k >> 1)] = pack_bf16(e[0], e[1]);
-          pk[hf * 32 + (k >> 1) + 1] = pack_bf16(e[2], e[3]);
-        }
+        if (full) key_half<true>(v, nl_w, c, key_ok, qmin, cs8, pk);
+        else key_half<false>(v, nl_w, c, key_ok, qmin, cs8, pk);
       }
-      const float cs = ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
-      if (key_ok && head_ok) part[cache ? key : M + key] = cs;
-      // P^T row r -> query blocks 2w, 2w + 1, once the previous O^T MMA is done
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
-                                             p.err, kWaitLimitNs, kErrTimeout));
-      if (!ok) break;
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const uint32_t addr = p_row + (uint32_t)(ch >> 3) * kAtom +
-                              ((((uint32_t)ch & 7u) ^ (uint32_t)(r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[ch * 4]),
-                     "r"(pk[ch * 4 + 1]), "r"(pk[ch * 4 + 2]), "r"(pk[ch * 4 + 3])
-                     : "memory");
+      {
+        uint32_t v[2][32];
+        tmem_ld32(st_tmem + 64, v[0]);
+        tmem_ld32(st_tmem + 96, v[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_ST_EMPTY));
+        // this warpgroup's P^T half of the previous tile has been read by its O^T MMA:
+        // store the first 64 queries now, the second half's exponentials overlap it
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
+                                               p.err, kWaitLimitNs, kErrTimeout));
+        if (!ok) break;
+        store_p_half(p_row, r, pk);
+        if (full) key_half<true>(v, nl_w + 64, c, key_ok, qmin - 64, cs8, pk);
+        else key_half<false>(v, nl_w + 64, c, key_ok, qmin - 64, cs8, pk);
+        store_p_half(p_row + kAtom, r, pk);
       }
       fence_async_smem();
       mbar_arrive(bar(B_P_FULL));
+      const float cs = ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
+      if (key_ok && head_ok) part[cache ? key : M + key] = cs;
     }
 
     // ----- epilogue: O^T (lane = d, columns = queries) -> out rows via shared memory
