@@ -137,11 +137,8 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    from h2o_kv_cache_b200.replicas import max_over_ranks as _max
+    return _max(x, world, device="cuda")
 
 
 def blas_threads():
@@ -227,6 +224,7 @@ def run_ours(args, cfg):
     world, rank, local = dist_setup(args.gpus)
     import h2o_kv_cache_b200 as h2o
     from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    from h2o_kv_cache_b200.replicas import aggregate_throughput, replica_stream_layer
     dev = torch.device("cuda", local if world > 1 else 0)
     n_needed = args.warmup + 2 * args.steps + 1     # device-timed steps, then host-buffer steps
     n_chunks = min(cfg.n_chunks, n_needed)
@@ -235,7 +233,7 @@ def run_ours(args, cfg):
     layers = []                                    # per layer: (cache, chunks)
     for layer in range(cfg.layers):
         # each replica (rank) has its own seeded streams
-        Q, K, V = gen_batch(cfg, layer + 1000 * rank, device=dev, T=T)
+        Q, K, V = gen_batch(cfg, replica_stream_layer(rank, layer), device=dev, T=T)
         chunks = split_chunks(Q, K, V, bounds)
         del Q, K, V
         cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype, device=dev)
@@ -289,7 +287,7 @@ def run_ours(args, cfg):
         barrier(world)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_s = max_over_ranks(sum(step_ms) / 1e3, world)
-    value = world * cfg.B * cfg.S * args.steps / total_s
+    value = aggregate_throughput(cfg.B * cfg.S * args.steps, world, total_s)
     attn_ms = statistics.mean(k[0] for k in kern_ms) / cfg.layers
     sel_ms = statistics.mean(k[1] + k[2] + k[3] for k in kern_ms) / cfg.layers
 
@@ -317,7 +315,7 @@ def run_ours(args, cfg):
         e2e_ev[i][1].record(stream)
     barrier(world)
     e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3, world)
-    e2e_value = world * cfg.B * cfg.S * args.steps / e2e_s
+    e2e_value = aggregate_throughput(cfg.B * cfg.S * args.steps, world, e2e_s)
 
     peaks = load_peaks()
     flops = 4 * cfg.d * pairs / (args.steps * cfg.layers)       # per attention launch
