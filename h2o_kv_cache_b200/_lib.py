@@ -27,6 +27,7 @@ SIGNATURES = {
     "h2o_read_kv": (_i32, [_vp, _vp, _vp, _vp]),
     "h2o_info": (_i32, [_vp, ctypes.POINTER(_i64)]),
     "h2o_set_profiling": (_i32, [_vp, _i32]),
+    "h2o_step_timings": (_i32, [_vp, _i32, ctypes.POINTER(ctypes.c_float), _i32]),
     "h2o_last_timings": (_i32, [_vp, ctypes.POINTER(ctypes.c_float), _i32]),
     "h2o_destroy": (_i32, [_vp]),
     "h2o_last_error": (ctypes.c_char_p, [_vp]),

@@ -46,17 +46,20 @@ struct h2o_ctx {
   void* vc = nullptr;
   float* scores = nullptr;
   int32_t* pos = nullptr;
+  // device error word: mapped pinned host memory, so kernels report into it
+  // directly and no copy is enqueued per step; nonzero only after an error
   int* err = nullptr;
   DevBuf partials, newscore, freed;
   // staging for host pointers
   DevBuf st_q, st_k, st_v, st_out;
-  int* h_err = nullptr;  // pinned mirror of *err
-  cudaEvent_t err_ev = nullptr;
+  cudaEvent_t err_ev = nullptr;   // recorded after each step
   bool err_pending = false;
 
+  // per-kernel timing: a ring of event sets, one set per profiled step
+  static constexpr int kProfRing = 64;
   bool prof = false;
-  cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
-  bool ev_valid = false;
+  cudaEvent_t ev[kProfRing][5] = {};
+  int64_t prof_steps = 0;   // profiled steps recorded so far
 
   std::string msg = "no error";
 };
@@ -135,11 +138,10 @@ int check_device_error(h2o_ctx* h, bool wait) {
     if (e != cudaSuccess) return cuda_fail(h, e, "kernel execution");
   }
   h->err_pending = false;
-  const int w = *h->h_err;
+  const int w = *static_cast<volatile int*>(h->err);
   if (w == 0) return H2O_OK;
   // report once: clear the word so the handle's next step starts clean
-  *h->h_err = 0;
-  cudaMemset(h->err, 0, sizeof(int));
+  *static_cast<volatile int*>(h->err) = 0;
   if (w & h2o::kErrTimeout)
     return fail(h, H2O_ETIMEOUT, "a bounded in-kernel wait timed out (device error word 0x%x)", w);
   if (w & h2o::kErrSelect)
@@ -205,7 +207,8 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   H2O_CUDA(h, ensure(h->newscore, (size_t)BH * S * sizeof(float)), "scratch alloc");
   H2O_CUDA(h, ensure(h->freed, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
 
-  if (h->prof) H2O_CUDA(h, cudaEventRecord(h->ev[0], st), "event");
+  cudaEvent_t* evs = h->ev[h->prof_steps % h2o_ctx::kProfRing];
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[0], st), "event");
 
   h2o::AttnArgs a;
   a.q = dq;
@@ -227,33 +230,32 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   if (fault_injected("launch")) return fail(h, H2O_ECUDA, "injected launch failure");
   cudaError_t e = h->use_umma ? h2o::launch_attn_umma(a, st) : h2o::launch_attn_simt(a, h->dtype, st);
   if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
-  if (h->prof) H2O_CUDA(h, cudaEventRecord(h->ev[1], st), "event");
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[1], st), "event");
 
   e = h2o::launch_score_reduce(static_cast<float*>(h->partials.p), h->scores,
                                static_cast<float*>(h->newscore.p), BH, h->G, S, h->M,
                                h->n_valid, h->row_tile, st);
   if (e != cudaSuccess) return cuda_fail(h, e, "score reduce launch");
-  if (h->prof) H2O_CUDA(h, cudaEventRecord(h->ev[2], st), "event");
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[2], st), "event");
 
   e = h2o::launch_select(h->scores, h->pos, BH, h->M, h->t0, h->R, need, h->n_valid, S,
                          static_cast<int32_t*>(h->freed.p), S, h->err, st);
   if (e != cudaSuccess) return cuda_fail(h, e, "select launch");
-  if (h->prof) H2O_CUDA(h, cudaEventRecord(h->ev[3], st), "event");
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[3], st), "event");
 
   e = h2o::launch_scatter(dk, dv, h->kc, h->vc, h->scores, h->pos,
                           static_cast<int32_t*>(h->freed.p), static_cast<float*>(h->newscore.p),
                           BH, S, h->M, h->d, (int)es, h->t0, st);
   if (e != cudaSuccess) return cuda_fail(h, e, "scatter launch");
   if (h->prof) {
-    H2O_CUDA(h, cudaEventRecord(h->ev[4], st), "event");
-    h->ev_valid = true;
+    H2O_CUDA(h, cudaEventRecord(evs[4], st), "event");
+    ++h->prof_steps;
   }
   h->last_launches = 4;
 
   if (hout) H2O_CUDA(h, cudaMemcpyAsync(out, dout, q_bytes, cudaMemcpyDefault, st), "copy out");
 
-  // error word: async read-back, checked by the next call
-  H2O_CUDA(h, cudaMemcpyAsync(h->h_err, h->err, sizeof(int), cudaMemcpyDeviceToHost, st), "err copy");
+  // the error word is read once this event has completed (by the next call)
   H2O_CUDA(h, cudaEventRecord(h->err_ev, st), "event");
   h->err_pending = true;
 
@@ -275,16 +277,20 @@ int alloc_state(h2o_ctx* h, int B) {
   H2O_CUDA(h, dev_alloc(&h->vc, slots * h->d * es), "cache alloc");
   H2O_CUDA(h, dev_alloc((void**)&h->scores, slots * sizeof(float)), "state alloc");
   H2O_CUDA(h, dev_alloc((void**)&h->pos, slots * sizeof(int32_t)), "state alloc");
-  H2O_CUDA(h, dev_alloc((void**)&h->err, sizeof(int)), "state alloc");
+  {
+    void* hp = nullptr;
+    if (fault_injected("alloc")) return cuda_fail(h, cudaErrorMemoryAllocation, "state alloc");
+    H2O_CUDA(h, cudaHostAlloc(&hp, sizeof(int), cudaHostAllocMapped), "pinned alloc");
+    h->err = static_cast<int*>(hp);
+    *h->err = 0;
+  }
   H2O_CUDA(h, cudaMemset(h->kc, 0, slots * h->d * es), "memset");
   H2O_CUDA(h, cudaMemset(h->vc, 0, slots * h->d * es), "memset");
   H2O_CUDA(h, cudaMemset(h->scores, 0, slots * sizeof(float)), "memset");
   H2O_CUDA(h, cudaMemset(h->pos, 0xFF, slots * sizeof(int32_t)), "memset");
-  H2O_CUDA(h, cudaMemset(h->err, 0, sizeof(int)), "memset");
-  H2O_CUDA(h, cudaMallocHost((void**)&h->h_err, sizeof(int)), "pinned alloc");
-  *h->h_err = 0;
   H2O_CUDA(h, cudaEventCreateWithFlags(&h->err_ev, cudaEventDisableTiming), "event");
-  for (auto& ev : h->ev) H2O_CUDA(h, cudaEventCreate(&ev), "event");
+  for (auto& set : h->ev)
+    for (auto& ev : set) H2O_CUDA(h, cudaEventCreate(&ev), "event");
   H2O_CUDA(h, cudaDeviceSynchronize(), "state init");
   h->B = B;
   return H2O_OK;
@@ -398,18 +404,26 @@ int h2o_set_profiling(h2o_t h, int on) {
   if (!h) return fail(nullptr, H2O_EINVAL, "h2o_set_profiling: NULL handle");
   if (on && !h->prefilled) return fail(h, H2O_ESTATE, "h2o_set_profiling: prefill first");
   h->prof = on != 0;
-  h->ev_valid = false;
+  h->prof_steps = 0;
   return H2O_OK;
+}
+
+int h2o_step_timings(h2o_t h, int age, float* ms, int n) {
+  if (!h || (!ms && n > 0)) return fail(h, H2O_EINVAL, "h2o_step_timings: NULL argument");
+  if (age < 0 || age >= h2o_ctx::kProfRing || age >= h->prof_steps)
+    return fail(h, H2O_ESTATE, "h2o_step_timings: no profiled step of age %d", age);
+  cudaEvent_t* evs = h->ev[(h->prof_steps - 1 - age) % h2o_ctx::kProfRing];
+  H2O_CUDA(h, cudaEventSynchronize(evs[4]), "event sync");
+  int w = 0;
+  for (int i = 0; i < 4 && w < n; ++i, ++w)
+    H2O_CUDA(h, cudaEventElapsedTime(&ms[i], evs[i], evs[i + 1]), "event time");
+  return w;
 }
 
 int h2o_last_timings(h2o_t h, float* ms, int n) {
   if (!h || (!ms && n > 0)) return fail(h, H2O_EINVAL, "h2o_last_timings: NULL argument");
-  if (!h->ev_valid) return fail(h, H2O_ESTATE, "h2o_last_timings: no profiled step");
-  H2O_CUDA(h, cudaEventSynchronize(h->ev[4]), "event sync");
-  int w = 0;
-  for (int i = 0; i < 4 && w < n; ++i, ++w)
-    H2O_CUDA(h, cudaEventElapsedTime(&ms[i], h->ev[i], h->ev[i + 1]), "event time");
-  return w;
+  if (h->prof_steps == 0) return fail(h, H2O_ESTATE, "h2o_last_timings: no profiled step");
+  return h2o_step_timings(h, 0, ms, n);
 }
 
 int h2o_destroy(h2o_t h) {
@@ -422,13 +436,13 @@ int h2o_destroy(h2o_t h) {
   cudaFree(h->vc);
   cudaFree(h->scores);
   cudaFree(h->pos);
-  cudaFree(h->err);
+  if (h->err) cudaFreeHost(h->err);
   for (DevBuf* b : {&h->partials, &h->newscore, &h->freed, &h->st_q, &h->st_k, &h->st_v, &h->st_out})
     cudaFree(b->p);
-  if (h->h_err) cudaFreeHost(h->h_err);
   if (h->err_ev) cudaEventDestroy(h->err_ev);
-  for (auto ev : h->ev)
-    if (ev) cudaEventDestroy(ev);
+  for (auto& set : h->ev)
+    for (auto ev : set)
+      if (ev) cudaEventDestroy(ev);
   delete h;
   return H2O_OK;
 }

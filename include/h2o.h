@@ -116,12 +116,18 @@ int h2o_read_kv(h2o_t h, void* k_cache, void* v_cache, void* stream);
  * device kernels launched by the last step (or prefill).                      */
 int h2o_info(h2o_t h, int64_t out[5]);
 
-/* Per-kernel timing.  When on (default off), each step records CUDA events
- * around its kernels on the caller's stream; h2o_last_timings() waits for the
- * last step's events and writes up to n durations in milliseconds:
+/* Per-kernel timing.  When on (default off; turning it on restarts the count),
+ * each step records CUDA events around its kernels on the caller's stream,
+ * into a ring that holds the last 64 steps, so steps can be enqueued back to
+ * back and read afterwards.  h2o_step_timings() waits for the events of the
+ * step `age` steps before the last (age 0 = the last step) and writes up to n
+ * durations in milliseconds:
  *   ms[0] attention + summed weights, ms[1] score accumulate, ms[2] select,
- *   ms[3] scatter.  Returns the number written (>= 0) or a negative status. */
+ *   ms[3] scatter.  Returns the number written (>= 0) or a negative status
+ *   (H2O_ESTATE if no such profiled step).  h2o_last_timings(h, ms, n) is
+ *   h2o_step_timings(h, 0, ms, n).                                            */
 int h2o_set_profiling(h2o_t h, int on);
+int h2o_step_timings(h2o_t h, int age, float* ms, int n);
 int h2o_last_timings(h2o_t h, float* ms, int n);
 
 /* Free every resource of the handle (synchronises the device first).  NULL is
