@@ -277,7 +277,7 @@ def run_ours(args, cfg):
             launches += sum(c.info()["launches"] for c, _ in layers)
         barrier(world)
     for i in range(args.steps):
-        t = [0.0, 0.0, 0.0, 0.0]
+        t = [0.0, 0.0]
         for cache, _ in layers:
             t = [a + b for a, b in zip(t, cache.last_timings(age=args.steps - 1 - i))]
         kern_ms.append(t)
@@ -285,7 +285,7 @@ def run_ours(args, cfg):
     total_s = max_over_ranks(sum(step_ms) / 1e3, world)
     value = aggregate_throughput(cfg.B * cfg.S * args.steps, world, total_s)
     attn_ms = statistics.mean(k[0] for k in kern_ms) / cfg.layers
-    sel_ms = statistics.mean(k[1] + k[2] + k[3] for k in kern_ms) / cfg.layers
+    sel_ms = statistics.mean(k[1] for k in kern_ms) / cfg.layers
 
     # end to end through the C ABI with host buffers (pinned), copies inside the region
     for cache, _ in layers:
@@ -350,9 +350,7 @@ def run_ours(args, cfg):
         "gpu_launches": launches,
         "clocks": clocks.summary(),
         "kernel_ms_per_layer": {"attention": attn_ms,
-                                "score_reduce": statistics.mean(k[1] for k in kern_ms) / cfg.layers,
-                                "select": statistics.mean(k[2] for k in kern_ms) / cfg.layers,
-                                "scatter": statistics.mean(k[3] for k in kern_ms) / cfg.layers},
+                                "tail (score accumulate + select + scatter)": sel_ms},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         chunks0 = layers[0][1]

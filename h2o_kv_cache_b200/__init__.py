@@ -131,10 +131,10 @@ class H2OCache:
         self._chk(lib.h2o_set_profiling(self._h, 1 if on else 0))
 
     def last_timings(self, age: int = 0):
-        """ms of [attention, score accumulate, select, scatter] of the profiled
-        step `age` steps before the last (0 = the last; up to 63)."""
-        arr = (ctypes.c_float * 4)()
-        n = lib.h2o_step_timings(self._h, age, arr, 4)
+        """ms of [attention, tail (score accumulate + select + scatter)] of the
+        profiled step `age` steps before the last (0 = the last; up to 63)."""
+        arr = (ctypes.c_float * 2)()
+        n = lib.h2o_step_timings(self._h, age, arr, 2)
         if n < 0:
             self._chk(n)
         return list(arr)[:n]

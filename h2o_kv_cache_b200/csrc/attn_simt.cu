@@ -52,7 +52,10 @@ __global__ void __launch_bounds__(BR) attn_simt_kernel(AttnArgs a) {
   const T* vb = static_cast<const T*>(a.v) + ((int64_t)b * a.Hkv + h) * S * D;
   const T* kcb = static_cast<const T*>(a.kc) + ((int64_t)b * a.Hkv + h) * M * D;
   const T* vcb = static_cast<const T*>(a.vc) + ((int64_t)b * a.Hkv + h) * M * D;
-  float* part = a.partials + (((int64_t)b * a.Hkv + h) * (G * n_rt) + (gl * n_rt + rt)) * (M + S);
+  float* part = a.partials + (((int64_t)b * a.Hkv + h) * (G * n_rt) + (gl * n_rt + rt)) * a.part_stride;
+
+  // the cache and the partial rows may still be in use by the previous kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   for (int e = tid; e < BR * D; e += BR) {
     const int r = e / D, c = e - r * D;
@@ -138,25 +141,33 @@ __global__ void __launch_bounds__(BR) attn_simt_kernel(AttnArgs a) {
 }
 
 template <typename T, int D>
-cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_t(const AttnArgs& a, bool pdl, cudaStream_t st) {
   const size_t smem = sizeof(float) * (BR * (D + 1) + 2 * BK * D + BR * (BK + 1));
   auto kern = attn_simt_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((a.S + BR - 1) / BR), (unsigned)a.Hq, (unsigned)a.B);
-  kern<<<grid, BR, smem, st>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((a.S + BR - 1) / BR), (unsigned)a.Hq, (unsigned)a.B);
+  cfg.blockDim = dim3(BR);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace
 
-cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t st) {
+cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, bool pdl, cudaStream_t st) {
   if (dtype == kF32) {
-    if (a.d == 64) return launch_t<float, 64>(a, st);
-    if (a.d == 128) return launch_t<float, 128>(a, st);
+    if (a.d == 64) return launch_t<float, 64>(a, pdl, st);
+    if (a.d == 128) return launch_t<float, 128>(a, pdl, st);
   } else {
-    if (a.d == 64) return launch_t<__nv_bfloat16, 64>(a, st);
-    if (a.d == 128) return launch_t<__nv_bfloat16, 128>(a, st);
+    if (a.d == 64) return launch_t<__nv_bfloat16, 64>(a, pdl, st);
+    if (a.d == 128) return launch_t<__nv_bfloat16, 128>(a, pdl, st);
   }
   return cudaErrorInvalidValue;
 }

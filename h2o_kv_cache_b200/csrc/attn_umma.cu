@@ -61,7 +61,8 @@ constexpr uint32_t kOffLse = kOffR + kRBytes;           // negated base-2 lse, [
 constexpr uint32_t kOffBar = kOffLse + 2 * BM * 4;
 constexpr int kNumBars = 24;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmemUsed = kOffMisc + 16;
+constexpr uint32_t kOffCs = kOffMisc + 16;             // head B's column sums of a tile, [128]
+constexpr uint32_t kSmemUsed = kOffCs + BN * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // slack for 1024-byte alignment
 static_assert(2 * kSlot1 <= kRBytes, "sweep-1 slots fit in R");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -71,15 +72,16 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;     // 1 s per wait
 enum { B_Q = 0, B_R1_FULL = 1, B_R1_EMPTY = 3, B_R2_FULL = 5, B_R2_EMPTY = B_R2_FULL + NS2,
        B_S_FULL = B_R2_EMPTY + NS2, B_S_EMPTY = B_S_FULL + 2, B_ST_FULL = B_S_EMPTY + 2,
        B_ST_EMPTY = B_ST_FULL + 1, B_P_FULL = B_ST_EMPTY + 1, B_P_EMPTY = B_P_FULL + 1,
-       B_O_FULL = B_P_EMPTY + 1, B_DRAIN = B_O_FULL + 1 };
-static_assert(B_DRAIN < kNumBars, "barrier count");
+       B_O_FULL = B_P_EMPTY + 1, B_DRAIN = B_O_FULL + 1, B_CS_FULL = B_DRAIN + 1,
+       B_CS_EMPTY = B_CS_FULL + 1 };
+static_assert(B_CS_EMPTY < kNumBars, "barrier count");
 
 struct Params {
   float* partials;
   int* err;
   void* out;
   int B, Hq, Hkv, G, n_pg, n_rt;
-  int64_t S, M, n_valid;
+  int64_t S, M, n_valid, stride;   // stride: floats between partial rows
   float scale_log2;   // (1/sqrt(d)) * log2(e)
 };
 
@@ -192,6 +194,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       uint32_t cnt = 1;
       if (i == B_S_EMPTY || i == B_S_EMPTY + 1) cnt = 128;   // one warpgroup
       if (i == B_ST_EMPTY || i == B_P_FULL) cnt = 256;        // both warpgroups
+      if (i == B_CS_FULL || i == B_CS_EMPTY) cnt = 128;       // one warpgroup
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -205,6 +208,8 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the cache and the partial rows may still be in use by the previous kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // tile t (128 keys): tensor map and row offset
   auto tile_src = [&](int t, bool v, const CUtensorMap*& m, int& y) {
@@ -428,7 +433,13 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     named_bar_sync(1 + w, 128);
 
     // ----- sweep 2: thread = key (lane r of S^T), the 128 query columns of head w
-    float* part = p.partials + ((int64_t)bh * (p.G * p.n_rt) + ((gl_a + w) * p.n_rt + rt)) * (M + S);
+    // One partial row per (head pair, row tile): warpgroup 1 hands head B's
+    // column sum of each key to warpgroup 0 through cs_b, which stores the
+    // sum of the two (an exact two-term add) one tile later.
+    float* part = p.partials + ((int64_t)bh * (p.n_pg * p.n_rt) + (pg * p.n_rt + rt)) * p.stride;
+    float* cs_b = reinterpret_cast<float*>(sbase + kOffCs);
+    float prev_cs = 0.f;
+    int64_t prev_col = -1;
     const uint32_t p_row = base + kOffP + (uint32_t)(2 * w) * kAtom + (uint32_t)(r >> 3) * 1024u +
                            (uint32_t)(r & 7) * 128u;
     const float* nl_w = nlse + w * BM;
@@ -438,6 +449,14 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                              kWaitLimitNs, kErrTimeout));
       if (!ok) break;
       tc_fence_after();
+      if (w == 0 && j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_FULL), (uint32_t)(j - 1) & 1u, abort_flag,
+                                               p.err, kWaitLimitNs, kErrTimeout));
+        if (!ok) break;
+        const float other = cs_b[r];
+        mbar_arrive(bar(B_CS_EMPTY));
+        if (prev_col >= 0) part[prev_col] = prev_cs + other;
+      }
       const bool cache = j < nct;
       const int64_t key = cache ? (int64_t)j * BN + r : (int64_t)(j - nct) * BN + r;
       const bool key_ok = cache ? key < nv : key < S;
@@ -474,7 +493,22 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       fence_async_smem();
       mbar_arrive(bar(B_P_FULL));
       const float cs = ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
-      if (key_ok && head_ok) part[cache ? key : M + key] = cs;
+      if (w == 0) {
+        prev_cs = cs;
+        prev_col = key_ok ? (cache ? key : M + key) : -1;
+      } else {
+        // without a head B every probability of this warpgroup is 0
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
+                                               p.err, kWaitLimitNs, kErrTimeout));
+        if (!ok) break;
+        cs_b[r] = head_ok ? cs : 0.f;
+        mbar_arrive(bar(B_CS_FULL));
+      }
+    }
+    if (w == 0 && ok && n > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_FULL), (uint32_t)(n - 1) & 1u, abort_flag,
+                                             p.err, kWaitLimitNs, kErrTimeout));
+      if (ok && prev_col >= 0) part[prev_col] = prev_cs + cs_b[r];
     }
 
     // ----- epilogue: O^T (lane = d, columns = queries) -> out rows via shared memory
@@ -545,7 +579,7 @@ cudaError_t make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t z) {
 
 bool attn_umma_supported(int dtype, int d) { return dtype == kBF16 && d == D; }
 
-cudaError_t launch_attn_umma(const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_attn_umma(const AttnArgs& a, bool pdl, cudaStream_t st) {
   if (a.d != D) return cudaErrorInvalidValue;
   cudaError_t e = get_encode();
   if (e != cudaSuccess) return e;
@@ -571,12 +605,22 @@ cudaError_t launch_attn_umma(const AttnArgs& a, cudaStream_t st) {
   p.S = a.S;
   p.M = a.M;
   p.n_valid = a.n_valid;
+  p.stride = a.part_stride;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   e = cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const int64_t grid = BHkv * p.n_pg * p.n_rt;
-  attn_umma_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, mkc, mvc, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_umma_kernel, mq, mk, mv, mkc, mvc, p);
 }
 
 }  // namespace h2o

@@ -55,10 +55,15 @@ struct h2o_ctx {
   cudaEvent_t err_ev = nullptr;   // recorded after each step
   bool err_pending = false;
 
-  // per-kernel timing: a ring of event sets, one set per profiled step
+  // fused tail: cluster size for (M, tail_S), 0 = use the three separate kernels
+  int64_t tail_S = -1;
+  int tail_cs = 0;
+
+  // per-kernel timing: a ring of event sets (start, after attention, after the
+  // tail), one set per profiled step
   static constexpr int kProfRing = 64;
   bool prof = false;
-  cudaEvent_t ev[kProfRing][5] = {};
+  cudaEvent_t ev[kProfRing][3] = {};
   int64_t prof_steps = 0;   // profiled steps recorded so far
 
   std::string msg = "no error";
@@ -119,6 +124,13 @@ bool is_device_ptr(const void* p) {
     return false;
   }
   return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+// H2O_SPLIT_TAIL=1 runs score accumulation, selection and scatter as three
+// kernels instead of the fused cluster kernel (same results).
+bool split_tail() {
+  const char* s = getenv("H2O_SPLIT_TAIL");
+  return s && s[0] == '1';
 }
 
 bool sync_check_enabled() {
@@ -202,9 +214,10 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
 
   // scratch sized for this chunk
   const int n_rt = (int)((S + h->row_tile - 1) / h->row_tile);
-  const size_t part_bytes = (size_t)BH * h->G * n_rt * (h->M + S) * sizeof(float);
+  const int64_t stride = h2o::partial_stride(h->M, S);
+  const int n_grp = h2o::partial_groups(h->G, h->use_umma);
+  const size_t part_bytes = (size_t)BH * n_grp * n_rt * stride * sizeof(float);
   H2O_CUDA(h, ensure(h->partials, part_bytes), "scratch alloc");
-  H2O_CUDA(h, ensure(h->newscore, (size_t)BH * S * sizeof(float)), "scratch alloc");
   H2O_CUDA(h, ensure(h->freed, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
 
   cudaEvent_t* evs = h->ev[h->prof_steps % h2o_ctx::kProfRing];
@@ -226,32 +239,62 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   a.S = S;
   a.M = h->M;
   a.n_valid = h->n_valid;
+  a.part_stride = stride;
   a.scale = (float)(1.0 / std::sqrt((double)h->d));
   if (fault_injected("launch")) return fail(h, H2O_ECUDA, "injected launch failure");
-  cudaError_t e = h->use_umma ? h2o::launch_attn_umma(a, st) : h2o::launch_attn_simt(a, h->dtype, st);
+  cudaError_t e = h->use_umma ? h2o::launch_attn_umma(a, true, st)
+                               : h2o::launch_attn_simt(a, h->dtype, true, st);
   if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
   if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[1], st), "event");
 
-  e = h2o::launch_score_reduce(static_cast<float*>(h->partials.p), h->scores,
-                               static_cast<float*>(h->newscore.p), BH, h->G, S, h->M,
-                               h->n_valid, h->row_tile, st);
-  if (e != cudaSuccess) return cuda_fail(h, e, "score reduce launch");
-  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[2], st), "event");
-
-  e = h2o::launch_select(h->scores, h->pos, BH, h->M, h->t0, h->R, need, h->n_valid, S,
-                         static_cast<int32_t*>(h->freed.p), S, h->err, st);
-  if (e != cudaSuccess) return cuda_fail(h, e, "select launch");
-  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[3], st), "event");
-
-  e = h2o::launch_scatter(dk, dv, h->kc, h->vc, h->scores, h->pos,
-                          static_cast<int32_t*>(h->freed.p), static_cast<float*>(h->newscore.p),
-                          BH, S, h->M, h->d, (int)es, h->t0, st);
-  if (e != cudaSuccess) return cuda_fail(h, e, "scatter launch");
+  if (S != h->tail_S) {
+    h->tail_cs = split_tail() ? 0 : h2o::tail_cluster_size(h->M, S, BH);
+    h->tail_S = S;
+  }
+  if (h->tail_cs > 0) {
+    h2o::TailArgs t;
+    t.partials = static_cast<const float*>(h->partials.p);
+    t.scores = h->scores;
+    t.pos = h->pos;
+    t.k = static_cast<const uint4*>(dk);
+    t.v = static_cast<const uint4*>(dv);
+    t.kc = static_cast<uint4*>(h->kc);
+    t.vc = static_cast<uint4*>(h->vc);
+    t.freed = static_cast<int32_t*>(h->freed.p);
+    t.err = h->err;
+    t.M = h->M;
+    t.S = S;
+    t.n_valid = h->n_valid;
+    t.t0 = h->t0;
+    t.R = h->R;
+    t.need = need;
+    t.stride = stride;
+    t.n_grp = n_grp;
+    t.n_rt = n_rt;
+    t.row_tile = h->row_tile;
+    t.row_vecs = (int)(h->d * es / 16);
+    e = h2o::launch_tail(t, BH, h->tail_cs, true, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "tail launch");
+    h->last_launches = 2;
+  } else {
+    H2O_CUDA(h, ensure(h->newscore, (size_t)BH * S * sizeof(float)), "scratch alloc");
+    e = h2o::launch_score_reduce(static_cast<float*>(h->partials.p), h->scores,
+                                 static_cast<float*>(h->newscore.p), BH, n_grp, S, h->M,
+                                 h->n_valid, h->row_tile, stride, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "score reduce launch");
+    e = h2o::launch_select(h->scores, h->pos, BH, h->M, h->t0, h->R, need, h->n_valid, S,
+                           static_cast<int32_t*>(h->freed.p), S, h->err, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "select launch");
+    e = h2o::launch_scatter(dk, dv, h->kc, h->vc, h->scores, h->pos,
+                            static_cast<int32_t*>(h->freed.p), static_cast<float*>(h->newscore.p),
+                            BH, S, h->M, h->d, (int)es, h->t0, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "scatter launch");
+    h->last_launches = 4;
+  }
   if (h->prof) {
-    H2O_CUDA(h, cudaEventRecord(evs[4], st), "event");
+    H2O_CUDA(h, cudaEventRecord(evs[2], st), "event");
     ++h->prof_steps;
   }
-  h->last_launches = 4;
 
   if (hout) H2O_CUDA(h, cudaMemcpyAsync(out, dout, q_bytes, cudaMemcpyDefault, st), "copy out");
 
@@ -413,9 +456,9 @@ int h2o_step_timings(h2o_t h, int age, float* ms, int n) {
   if (age < 0 || age >= h2o_ctx::kProfRing || age >= h->prof_steps)
     return fail(h, H2O_ESTATE, "h2o_step_timings: no profiled step of age %d", age);
   cudaEvent_t* evs = h->ev[(h->prof_steps - 1 - age) % h2o_ctx::kProfRing];
-  H2O_CUDA(h, cudaEventSynchronize(evs[4]), "event sync");
+  H2O_CUDA(h, cudaEventSynchronize(evs[2]), "event sync");
   int w = 0;
-  for (int i = 0; i < 4 && w < n; ++i, ++w)
+  for (int i = 0; i < 2 && w < n; ++i, ++w)
     H2O_CUDA(h, cudaEventElapsedTime(&ms[i], evs[i], evs[i + 1]), "event time");
   return w;
 }

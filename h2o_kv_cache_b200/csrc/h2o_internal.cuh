@@ -19,11 +19,24 @@ enum : int {
 };
 
 // One chunk's attention with summed weights, for all (b, KV head) of a layer.
-// Column c of a partial row: c < M is cache slot c, c = M + j is chunk key j.
-// Partial row tq of a (b, h) group belongs to query-row tile (local head gl,
-// row tile rt): tq = gl * n_rt + rt, n_rt = ceil(S / row_tile).  A tile writes
-// every cache column < n_valid and the chunk columns of keys it can see
-// (key j < min(S, (rt + 1) * row_tile)).
+// Column c of a partial row: c < M is cache slot c, c = M + j is chunk key j;
+// rows are part_stride floats apart (M + S rounded up to a multiple of 4, so
+// every row starts 16-byte aligned).  Partial row tq of a (b, h) group belongs
+// to (group gl, row tile rt): tq = gl * n_rt + rt, n_rt = ceil(S / row_tile).
+// A group is one query head of the KV head's G in the SIMT kernel, and a pair
+// of them (heads 2gl and 2gl + 1, summed) in the tensor-core kernel; see
+// partial_groups().  A tile writes every cache column < n_valid and the chunk
+// columns of keys it can see (key j < min(S, (rt + 1) * row_tile)).
+inline int64_t partial_stride(int64_t M, int64_t S) { return (M + S + 3) & ~(int64_t)3; }
+inline int partial_groups(int G, bool umma) { return umma ? (G + 1) / 2 : G; }
+
+// Order in which a column's partial rows are added, shared by both tail paths
+// so they agree bit for bit: the column's list of n rows (for a chunk column,
+// the rows that wrote it, group-major) is cut into kQuarters contiguous runs,
+// run q = [q * n / kQuarters, (q + 1) * n / kQuarters); each run is summed in
+// order starting from 0, and then the run sums are added in order.
+constexpr int kQuarters = 4;
+
 struct AttnArgs {
   const void* q;      // [B, Hq, S, d]
   const void* k;      // [B, Hkv, S, d]
@@ -31,10 +44,10 @@ struct AttnArgs {
   void* out;          // [B, Hq, S, d] or nullptr
   const void* kc;     // [B, Hkv, M, d]
   const void* vc;     // [B, Hkv, M, d]
-  float* partials;    // [B, Hkv, G * n_rt, M + S]
+  float* partials;    // [B, Hkv, partial_groups * n_rt, part_stride]
   int* err;           // device error word
   int B, Hq, Hkv, d;
-  int64_t S, M, n_valid;
+  int64_t S, M, n_valid, part_stride;
   float scale;        // 1/sqrt(d)
 };
 
@@ -42,15 +55,18 @@ struct AttnArgs {
 constexpr int kSimtRowTile = 64;
 constexpr int kUmmaRowTile = 128;
 
-cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t st);
-cudaError_t launch_attn_umma(const AttnArgs& a, cudaStream_t st);
+// Both kernels wait (griddepcontrol.wait) before their first global access, so
+// with pdl they are launched as programmatic dependents of the stream's
+// previous kernel and their prologue overlaps its last blocks.
+cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, bool pdl, cudaStream_t st);
+cudaError_t launch_attn_umma(const AttnArgs& a, bool pdl, cudaStream_t st);
 bool attn_umma_supported(int dtype, int d);
 
 // scores[b,h,c] += sum of partial column c (c < n_valid);
-// newscore[b,h,j] = sum of partial column M + j (j < S).
+// newscore[b,h,j] = sum of partial column M + j (j < S); n_grp partial groups.
 cudaError_t launch_score_reduce(const float* partials, float* scores, float* newscore, int BH,
-                                int G, int64_t S, int64_t M, int64_t n_valid, int row_tile,
-                                cudaStream_t st);
+                                int n_grp, int64_t S, int64_t M, int64_t n_valid, int row_tile,
+                                int64_t part_stride, cudaStream_t st);
 
 // freed[bh, 0..S) = ascending evicted slots (need of them), then empty slots
 // n_valid, n_valid + 1, ...  Sets kErrSelect in *err if a head has too few
@@ -63,6 +79,27 @@ cudaError_t launch_select(const float* scores, const int32_t* pos, int BH, int64
 cudaError_t launch_scatter(const void* k, const void* v, void* kc, void* vc, float* scores,
                            int32_t* pos, const int32_t* freed, const float* newscore, int BH,
                            int64_t S, int64_t M, int d, int esize, int64_t t0, cudaStream_t st);
+
+// The three steps above as one launch: one thread-block cluster per (b, KV
+// head).  freed[bh, 0..S) gets the same list launch_select writes.
+struct TailArgs {
+  const float* partials;   // [BH, n_grp * n_rt, stride]
+  float* scores;           // [BH, M]
+  int32_t* pos;            // [BH, M]
+  const uint4* k;          // chunk keys [BH, S, row_vecs]
+  const uint4* v;          // chunk values [BH, S, row_vecs]
+  uint4* kc;               // cache keys [BH, M, row_vecs]
+  uint4* vc;               // cache values [BH, M, row_vecs]
+  int32_t* freed;          // [BH, S]
+  int* err;
+  int64_t M, S, n_valid, t0, R, need, stride;
+  int n_grp, n_rt, row_tile, row_vecs;
+  int per, per_s;          // set by launch_tail
+};
+// Cluster size the fused tail runs with for these sizes (16, 8, ..., 1), or 0
+// if it cannot run (the caller then uses the three separate kernels).
+int tail_cluster_size(int64_t M, int64_t S, int BH);
+cudaError_t launch_tail(const TailArgs& a, int BH, int cs, bool pdl, cudaStream_t st);
 
 // Records msg as this thread's last error (h2o_last_error(NULL)); returns code.
 int set_thread_error(int code, const char* msg);

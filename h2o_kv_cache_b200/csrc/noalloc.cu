@@ -58,22 +58,22 @@ cudaError_t scratch_address(void** out) {
 // colsum[bh, M + j]: chunk key j's summed weight.  Fixed-order sums of the
 // attention kernel's partial rows.
 __global__ void colsum_kernel(const float* __restrict__ partials, float* __restrict__ colsum, int G,
-                              int64_t S, int64_t M, int64_t n_valid, int row_tile) {
+                              int64_t S, int64_t M, int64_t n_valid, int row_tile, int64_t stride) {
   const int bh = blockIdx.y;
   const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t ncol = M + S;
   if (c >= ncol) return;
   const int n_rt = (int)((S + row_tile - 1) / row_tile);
-  const float* base = partials + (int64_t)bh * (G * n_rt) * ncol;
+  const float* base = partials + (int64_t)bh * (G * n_rt) * stride;
   float acc = 0.f;
   if (c < M) {
     if (c < n_valid)
-      for (int t = 0; t < G * n_rt; ++t) acc += base[(int64_t)t * ncol + c];
+      for (int t = 0; t < G * n_rt; ++t) acc += base[(int64_t)t * stride + c];
   } else {
     const int64_t j = c - M;
     const int rt0 = (int)(j / row_tile);
     for (int gl = 0; gl < G; ++gl)
-      for (int rt = rt0; rt < n_rt; ++rt) acc += base[(int64_t)(gl * n_rt + rt) * ncol + c];
+      for (int rt = rt0; rt < n_rt; ++rt) acc += base[(int64_t)(gl * n_rt + rt) * stride + c];
   }
   colsum[(int64_t)bh * ncol + c] = acc;
 }
@@ -93,12 +93,13 @@ extern "C" int h2o_attend_noalloc(const void* q, const void* k, const void* v, c
   const int row_tile = umma ? h2o::kUmmaRowTile : h2o::kSimtRowTile;
   const int G = Hq / Hkv;
   const int64_t n_rt = (S + row_tile - 1) / row_tile;
-  const double need = (double)B * Hkv * G * n_rt * (double)(M + S);
+  const int64_t stride = h2o::partial_stride(M, S);
+  const double need = (double)B * Hkv * G * n_rt * (double)stride;
   if (need > (double)kScratchFloats) {
     char msg[256];
     snprintf(msg, sizeof(msg),
              "problem needs %.0f scratch floats, above the fixed maximum of %zu "
-             "(B*Hkv*(Hq/Hkv)*ceil(S/%d)*(M+S) must be <= %zu)",
+             "(B*Hkv*(Hq/Hkv)*ceil(S/%d)*(M+S rounded up to a multiple of 4) must be <= %zu)",
              need, kScratchFloats, row_tile, kScratchFloats);
     return set_err(H2O_ESHAPE, msg);
   }
@@ -130,12 +131,14 @@ extern "C" int h2o_attend_noalloc(const void* q, const void* k, const void* v, c
   a.S = S;
   a.M = M;
   a.n_valid = n_valid;
+  a.part_stride = stride;
   a.scale = (float)(1.0 / std::sqrt((double)d));
-  e = umma ? h2o::launch_attn_umma(a, st) : h2o::launch_attn_simt(a, dtype, st);
+  e = umma ? h2o::launch_attn_umma(a, false, st) : h2o::launch_attn_simt(a, dtype, false, st);
   if (e != cudaSuccess) return set_err(H2O_ECUDA, cudaGetErrorString(e));
   const int threads = 256;
   dim3 grid((unsigned)((M + S + threads - 1) / threads), (unsigned)(B * Hkv));
-  colsum_kernel<<<grid, threads, 0, st>>>(partials, colsum, G, S, M, n_valid, row_tile);
+  colsum_kernel<<<grid, threads, 0, st>>>(partials, colsum, h2o::partial_groups(G, umma), S, M,
+                                           n_valid, row_tile, stride);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_err(H2O_ECUDA, cudaGetErrorString(e));
   return H2O_OK;

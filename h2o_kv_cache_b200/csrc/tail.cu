@@ -1,0 +1,504 @@
+// The step's tail in one launch: score accumulation, masked selection of the
+// slots to evict, and the scatter of the chunk's K/V into the freed slots.
+//
+// "Learning how to Forget: Fine-tuning for Long-Context Sparse Attention",
+// §1 Introduction ¶1 (fixed-size cache, slots evicted once full) and ¶4 (H2O:
+// the running sum of summed attention weights ranks the slots); Figure 1(c)
+// (per-chunk buffer deltas: the evicted slots and the new K/V rows written
+// into them).
+//
+// One thread-block cluster per (b, KV head); CTA `rank` of the cluster owns
+// cache slots [rank * per, (rank + 1) * per) and chunk rows
+// [rank * per_s, (rank + 1) * per_s).  Phases, separated by cluster barriers:
+//   1. add the partial rows of the summed weights to the scores of its slots
+//      (fixed row order, so the result does not depend on scheduling), and
+//      form each eligible slot's 64-bit key (order-preserving score bits,
+//      token position) in shared memory; reduce the chunk columns of its rows
+//      into the new tokens' initial scores;
+//   2. MSD radix select, 11 bits a pass: every CTA adds its digit counts into
+//      rank 0's histogram through distributed shared memory, then all CTAs
+//      read the merged histogram and take the same decision;
+//   3. ordered compaction: per-CTA counts are exchanged through rank 0, and
+//      each CTA writes its evicted slots at its offset, ascending;
+//   4. scatter of the CTA's chunk rows into the freed slots (the rows are read
+//      at the start, so only the stores remain here).
+#include <cstdint>
+
+#include "h2o_internal.cuh"
+
+namespace h2o {
+namespace {
+
+constexpr int kTailThreads = 512;
+constexpr int kMaxCluster = 16;
+constexpr uint64_t kNoKey = ~0ull;   // ineligible slot (a real key has pos < 2^31)
+constexpr int kLanes = kTailThreads / kQuarters;   // columns (float4 or float) per round
+constexpr int kDigitBits = 11;                     // radix digit
+constexpr int kBins = 1 << kDigitBits;
+constexpr int kBinsPerThread = kBins / kTailThreads;
+static_assert(kBinsPerThread == 4, "one 16-byte histogram read per thread");
+constexpr int kPre = 8;                            // chunk rows per warp read ahead
+
+__device__ __forceinline__ void add4(float4& a, const float4 b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of `p` (a shared variable of this CTA) in the CTA of cluster rank `rank`.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void dsmem_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 dsmem_ld4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void dsmem_st(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ int32_t ld_relaxed(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ordered_bits(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix sum over the block; returns this thread's offset, *total
+// gets the block's sum.  Every thread must call it.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t* warp_sum, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  uint32_t before = 0, all = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+    const uint32_t s = warp_sum[w];
+    before += (w < warp) ? s : 0u;
+    all += s;
+  }
+  __syncthreads();   // warp_sum may be reused right after
+  *total = all;
+  return before + incl - x;
+}
+
+__global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
+  extern __shared__ __align__(16) unsigned char dyn[];
+  uint64_t* keys = reinterpret_cast<uint64_t*>(dyn);                   // [per]
+  float* ns = reinterpret_cast<float*>(dyn + (size_t)p.per * 8);       // [per_s]
+  __shared__ __align__(16) uint32_t hist[3][kBins];   // rank 0's copy is the merged one
+  __shared__ __align__(16) uint32_t hloc[kBins];      // this CTA's counts of a pass
+  __shared__ uint32_t cnt[kMaxCluster];               // rank 0: selected slots per rank
+  __shared__ uint32_t warp_sum[kTailThreads / 32];
+  __shared__ float4 red4[kQuarters - 1][kLanes];      // quarter sums 1..3 of slot columns
+  __shared__ float red1[kQuarters - 1][kLanes];       // ... and of chunk columns
+  __shared__ uint64_t sh_prefix, sh_mask;
+  __shared__ int64_t sh_kth;
+  __shared__ int sh_state;                            // 0 searching, 1 found, 2 too few
+  __shared__ uint32_t sh_off, sh_tot;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthr = kTailThreads, nwarps = kTailThreads / 32;
+  const uint32_t rank = cluster_rank(), cs = cluster_size();
+  const int64_t bh = blockIdx.x / cs;
+  const int64_t M = p.M, S = p.S, nv = p.n_valid, need = p.need;
+  const int64_t lo = (int64_t)rank * p.per, hi = lo + p.per < M ? lo + p.per : M;
+  const int64_t nloc = hi > lo ? hi - lo : 0;
+  const int64_t lo_s = (int64_t)rank * p.per_s, hi_s = lo_s + p.per_s < S ? lo_s + p.per_s : S;
+
+  if (rank == 0)
+    for (int i = tid; i < 2 * kBins; i += nthr) (&hist[0][0])[i] = 0u;
+  if (tid == 0) {
+    sh_prefix = 0;
+    sh_mask = 0;
+    sh_kth = need;
+    sh_state = need == 0 ? 1 : 0;
+  }
+  // everything below reads what the preceding kernel of the stream wrote
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // Chunk rows i = lo_s + warp + k * nwarps (k = 0, 1, ...) are this warp's to
+  // scatter.  The first kPre are read now, so that their latency hides behind
+  // the reduction and the selection: lane c holds vector c of the row's K
+  // vectors followed by its V vectors.
+  const int rv = p.row_vecs, vecs2 = 2 * rv;
+  const bool pre_ok = vecs2 <= 32;
+  const int64_t n_mine = hi_s - lo_s > warp ? (hi_s - lo_s - warp + nwarps - 1) / nwarps : 0;
+  uint4 pre[kPre];
+  if (pre_ok) {
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+      if (k < n_mine && lane < vecs2) {
+        const int64_t src = (bh * S + lo_s + warp + (int64_t)k * nwarps) * rv;
+        pre[k] = lane < rv ? __ldg(p.k + src + lane) : __ldg(p.v + src + lane - rv);
+      }
+    }
+  }
+
+  // ---- 1. scores += partial column sums; keys of the eligible slots; the
+  // chunk rows' initial scores.  A column's partial rows are added in the
+  // kQuarters-run order, here one thread a run; a round covers 4 * kLanes
+  // slots and kLanes chunk columns.
+  const int n_rows = p.n_grp * p.n_rt;
+  const float* base = p.partials + bh * (int64_t)n_rows * p.stride;
+  float* sc = p.scores + bh * M;
+  const int32_t* ps = p.pos + bh * M;
+  const int64_t lim = p.t0 - p.R;               // eligible: 0 <= pos < t0 - R
+  const int qr = tid / kLanes, ln = tid - qr * kLanes;
+  const int64_t s_end = hi < nv ? hi : nv;      // slots with partial columns
+  const int64_t n_sr = (nloc + 4 * kLanes - 1) / (4 * kLanes);
+  const int64_t n_cr = hi_s > lo_s ? (hi_s - lo_s + kLanes - 1) / kLanes : 0;
+  const int64_t rounds = n_sr > n_cr ? n_sr : n_cr;
+  for (int64_t rd = 0; rd < rounds; ++rd) {
+    const int64_t s0 = lo + rd * 4 * kLanes + 4 * ln;
+    float scv[4] = {0.f, 0.f, 0.f, 0.f};
+    int32_t psv[4] = {-1, -1, -1, -1};
+    if (qr == 0) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (s0 + e < hi) {
+          scv[e] = sc[s0 + e];
+          psv[e] = ps[s0 + e];
+        }
+    }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (s0 < s_end) {
+      const float* col = base + s0;
+      const int r_hi = (qr + 1) * n_rows / kQuarters;
+      int r = qr * n_rows / kQuarters;
+      for (; r + 8 <= r_hi; r += 8) {
+        float4 x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = __ldg(reinterpret_cast<const float4*>(col + (int64_t)(r + u) * p.stride));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) add4(acc, x[u]);
+      }
+      for (; r < r_hi; ++r) add4(acc, __ldg(reinterpret_cast<const float4*>(col + (int64_t)r * p.stride)));
+    }
+    const int64_t i = lo_s + rd * kLanes + ln;
+    float cacc = 0.f;
+    if (i < hi_s) {
+      const int rt0 = (int)(i / p.row_tile);    // chunk key i is seen by row tiles rt >= rt0
+      const int span = p.n_rt - rt0;
+      const int n = p.n_grp * span;             // rows (group, rt >= rt0), group-major
+      const float* col = base + M + i;
+      const int t_hi = (qr + 1) * n / kQuarters;
+      int t = qr * n / kQuarters;
+      for (; t + 8 <= t_hi; t += 8) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int g = (t + u) / span, rt = rt0 + (t + u) - g * span;
+          x[u] = __ldg(col + (int64_t)(g * p.n_rt + rt) * p.stride);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cacc += x[u];
+      }
+      for (; t < t_hi; ++t) {
+        const int g = t / span, rt = rt0 + t - g * span;
+        cacc += __ldg(col + (int64_t)(g * p.n_rt + rt) * p.stride);
+      }
+    }
+    if (qr > 0) {
+      red4[qr - 1][ln] = acc;
+      red1[qr - 1][ln] = cacc;
+    }
+    __syncthreads();
+    if (qr == 0) {
+      add4(acc, red4[0][ln]);
+      add4(acc, red4[1][ln]);
+      add4(acc, red4[2][ln]);
+      const float add[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t s = s0 + e;
+        if (s >= hi) break;
+        float v = scv[e];
+        if (s < nv) {
+          v += add[e];
+          sc[s] = v;
+        }
+        const int32_t q = psv[e];
+        keys[s - lo] = (q >= 0 && q < lim) ? ((uint64_t)ordered_bits(v) << 32) | (uint32_t)q : kNoKey;
+      }
+      if (i < hi_s) ns[i - lo_s] = ((cacc + red1[0][ln]) + red1[1][ln]) + red1[2][ln];
+    }
+    __syncthreads();
+  }
+  cluster_sync();   // rank 0's histograms are zero, every CTA has its keys
+
+  // ---- 2. radix select of the need-th smallest key over the cluster,
+  // kDigitBits a pass from the top (the last pass takes the 9 bits left)
+  const uint32_t hist0 = dsmem_addr(&hist[0][0], 0);
+  int pass = 0;
+  for (int top = 64; top > 0; top -= kDigitBits, ++pass) {
+    if (sh_state != 0) break;                   // uniform: every CTA took the same decisions
+    const int shift = top > kDigitBits ? top - kDigitBits : 0;
+    const uint32_t dmask = (1u << (top - shift)) - 1u;
+    const uint64_t prefix = sh_prefix, mask = sh_mask;
+    const int64_t kth = sh_kth;
+    const uint32_t H = hist0 + (uint32_t)((pass % 3) * kBins * 4);
+    // counts of this CTA's keys in shared memory, then one remote add per
+    // non-empty bin into rank 0's histogram
+    for (int b = tid; b < kBins; b += nthr) hloc[b] = 0u;
+    __syncthreads();
+    for (int64_t j0 = 0; j0 < nloc; j0 += nthr) {
+      const int64_t j = j0 + tid;
+      const uint64_t key = j < nloc ? keys[j] : kNoKey;
+      const bool take = key != kNoKey && (key & mask) == prefix;
+      const uint32_t digit = (uint32_t)(key >> shift) & dmask;
+      const unsigned act = __ballot_sync(0xffffffffu, take);
+      if (take) {
+        const unsigned peers = __match_any_sync(act, digit);
+        if ((__ffs(peers) - 1) == lane) atomicAdd(&hloc[digit], (uint32_t)__popc(peers));
+      }
+    }
+    __syncthreads();
+    {
+      const uint4 c4 = *reinterpret_cast<const uint4*>(&hloc[kBinsPerThread * tid]);
+      const uint32_t cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+      for (int b = 0; b < kBinsPerThread; ++b)
+        if (cv[b] != 0u) dsmem_add(H + (uint32_t)(kBinsPerThread * tid + b) * 4u, cv[b]);
+    }
+    // the histogram of the next pass was last read before the previous barrier
+    if (rank == 0)
+      for (int b = tid; b < kBins; b += nthr) hist[(pass + 1) % 3][b] = 0u;
+    cluster_sync();
+    // thread t reads merged bins [kBinsPerThread * t, kBinsPerThread * (t + 1))
+    const uint4 h4 = dsmem_ld4(H + (uint32_t)tid * 16u);
+    const uint32_t hv[4] = {h4.x, h4.y, h4.z, h4.w};
+    const uint32_t sum = (h4.x + h4.y) + (h4.z + h4.w);
+    uint32_t total;
+    const uint32_t excl = block_excl_scan(sum, warp_sum, &total);
+    if ((int64_t)excl < kth && kth <= (int64_t)(excl + sum)) {
+      int64_t before = excl;
+#pragma unroll
+      for (int b = 0; b < kBinsPerThread; ++b) {
+        if (before < kth && kth <= before + (int64_t)hv[b]) {
+          const int64_t rem = kth - before;
+          sh_prefix = prefix | ((uint64_t)(kBinsPerThread * tid + b) << shift);
+          sh_mask = mask | ((uint64_t)dmask << shift);
+          sh_kth = rem;
+          if ((int64_t)hv[b] == rem) sh_state = 1;   // the whole bucket is evicted
+        }
+        before += hv[b];
+      }
+    }
+    if (tid == 0 && (int64_t)total < kth) sh_state = 2;
+    __syncthreads();
+  }
+
+  // ---- 3. evicted slots in ascending order, then the empty slots
+  const int state = sh_state;
+  const uint64_t prefix = sh_prefix, mask = sh_mask;
+  const bool do_sel = need > 0 && state == 1;
+  const int64_t run = (nloc + nthr - 1) / nthr;
+  const int64_t j0 = (int64_t)tid * run, j1 = j0 + run < nloc ? j0 + run : nloc;
+  uint32_t mine = 0;
+  if (do_sel)
+    for (int64_t j = j0; j < j1; ++j) {
+      const uint64_t key = keys[j];
+      mine += (key != kNoKey && (key & mask) <= prefix) ? 1u : 0u;
+    }
+  uint32_t cta_sel;
+  const uint32_t my_off = block_excl_scan(mine, warp_sum, &cta_sel);
+  const uint32_t cnt0 = dsmem_addr(&cnt[0], 0);
+  if (tid == 0) dsmem_st(cnt0 + rank * 4u, cta_sel);
+  cluster_sync();
+  if (warp == 0) {
+    const uint32_t x = lane < (int)cs ? dsmem_ld(cnt0 + (uint32_t)lane * 4u) : 0u;
+    const uint32_t off = __reduce_add_sync(0xffffffffu, lane < (int)rank ? x : 0u);
+    const uint32_t tot = __reduce_add_sync(0xffffffffu, x);
+    if (lane == 0) {
+      sh_off = off;
+      sh_tot = tot;
+    }
+  }
+  __syncthreads();
+  const bool sel_ok = need == 0 || (state == 1 && (int64_t)sh_tot == need);
+  int32_t* fr = p.freed + bh * S;
+  if (do_sel) {
+    int64_t o = (int64_t)sh_off + my_off;
+    for (int64_t j = j0; j < j1; ++j) {
+      const uint64_t key = keys[j];
+      if (key != kNoKey && (key & mask) <= prefix) {
+        if (o < need) fr[o] = (int32_t)(lo + j);
+        ++o;
+      }
+    }
+  }
+  if (rank == 0 && tid == 0 && !sel_ok) atomicOr(p.err, kErrSelect);
+  for (int64_t e = (int64_t)rank * nthr + tid; e < S - need; e += (int64_t)cs * nthr)
+    fr[need + e] = (int32_t)(nv + e);
+  cluster_sync();   // the freed list is complete; rank 0's shared memory is no longer read
+
+  // ---- 4. chunk row i -> slot fr[i]: K and V rows, pos = t0 + i, initial score
+  if (!sel_ok) return;
+  auto finish_row = [&](int64_t i, int32_t slot) {
+    if (lane == 0) {
+      p.pos[bh * M + slot] = (int32_t)(p.t0 + i);
+      p.scores[bh * M + slot] = ns[i - lo_s];
+    }
+  };
+  int64_t k_from = 0;
+  if (pre_ok) {
+    // lane k fetches the slot of the warp's k-th row
+    const int32_t my_slot = lane < n_mine ? ld_relaxed(fr + lo_s + warp + (int64_t)lane * nwarps) : -1;
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+      if (k < n_mine) {
+        const int64_t i = lo_s + warp + (int64_t)k * nwarps;
+        const int32_t slot = __shfl_sync(0xffffffffu, my_slot, k);
+        if (slot < 0 || slot >= M) {
+          if (lane == 0) atomicOr(p.err, kErrBounds);
+        } else {
+          const int64_t dst = (bh * M + slot) * rv;
+          if (lane < rv) p.kc[dst + lane] = pre[k];
+          else if (lane < vecs2) p.vc[dst + lane - rv] = pre[k];
+          finish_row(i, slot);
+        }
+      }
+    }
+    k_from = kPre;
+  }
+  for (int64_t k0 = k_from; k0 < n_mine; k0 += 32) {
+    const int32_t my_slot = k0 + lane < n_mine ? ld_relaxed(fr + lo_s + warp + (k0 + lane) * nwarps) : -1;
+    const int kn = n_mine - k0 < 32 ? (int)(n_mine - k0) : 32;
+    for (int jj = 0; jj < kn; ++jj) {
+      const int64_t i = lo_s + warp + (k0 + jj) * nwarps;
+      const int32_t slot = __shfl_sync(0xffffffffu, my_slot, jj);
+      if (slot < 0 || slot >= M) {
+        if (lane == 0) atomicOr(p.err, kErrBounds);
+        continue;
+      }
+      const int64_t src = (bh * S + i) * rv, dst = (bh * M + slot) * rv;
+      for (int c = lane; c < vecs2; c += 32) {   // K row then V row
+        if (c < rv) p.kc[dst + c] = __ldg(p.k + src + c);
+        else p.vc[dst + c - rv] = __ldg(p.v + src + c - rv);
+      }
+      finish_row(i, slot);
+    }
+  }
+}
+
+size_t tail_smem(int64_t M, int64_t S, int cs, int* per, int* per_s) {
+  const int64_t pr = ((M + cs - 1) / cs + 3) & ~(int64_t)3;
+  const int64_t prs = (S + cs - 1) / cs;
+  *per = (int)pr;
+  *per_s = (int)prs;
+  return (size_t)pr * 8 + (size_t)prs * 4;
+}
+
+constexpr size_t kTailSmemMax = 180 * 1024;   // plus about 41 KB static
+
+}  // namespace
+
+int tail_cluster_size(int64_t M, int64_t S, int BH) {
+  static_assert(kMaxCluster == 16, "cluster sizes below assume 16");
+  if (cudaFuncSetAttribute(tail_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  // the fewest waves of clusters (all BH at once if possible), then the
+  // largest cluster
+  int best = 0;
+  int64_t best_waves = INT64_MAX;
+  for (int cs = kMaxCluster; cs >= 1; cs >>= 1) {
+    if (cs > 1 && M < 32LL * cs) continue;       // at least 32 slots a CTA
+    int per, per_s;
+    const size_t smem = tail_smem(M, S, cs, &per, &per_s);
+    if (smem > kTailSmemMax) break;               // grows as cs falls: no smaller size fits
+    if (cudaFuncSetAttribute(tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+      cudaGetLastError();
+      break;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(BH * cs));
+    cfg.blockDim = dim3(kTailThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, tail_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    if (n < 1) continue;
+    const int64_t waves = (BH + n - 1) / n;
+    if (waves < best_waves) {
+      best_waves = waves;
+      best = cs;
+    }
+  }
+  return best;
+}
+
+cudaError_t launch_tail(const TailArgs& a0, int BH, int cs, bool pdl, cudaStream_t st) {
+  if (cs < 1 || cs > kMaxCluster || (cs & (cs - 1)) != 0) return cudaErrorInvalidValue;
+  TailArgs a = a0;
+  const size_t smem = tail_smem(a.M, a.S, cs, &a.per, &a.per_s);
+  if (smem > kTailSmemMax) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(BH * cs));
+  cfg.blockDim = dim3(kTailThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)cs;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, tail_kernel, a);
+}
+
+}  // namespace h2o

@@ -122,8 +122,10 @@ int h2o_info(h2o_t h, int64_t out[5]);
  * back and read afterwards.  h2o_step_timings() waits for the events of the
  * step `age` steps before the last (age 0 = the last step) and writes up to n
  * durations in milliseconds:
- *   ms[0] attention + summed weights, ms[1] score accumulate, ms[2] select,
- *   ms[3] scatter.  Returns the number written (>= 0) or a negative status
+ *   ms[0] attention + summed weights, ms[1] the tail: score accumulate,
+ *   select and scatter (one fused launch, or three kernels when the fused one
+ *   cannot run for these sizes or H2O_SPLIT_TAIL=1 is set in the environment).
+ *   Returns the number written (>= 0) or a negative status
  *   (H2O_ESTATE if no such profiled step).  h2o_last_timings(h, ms, n) is
  *   h2o_step_timings(h, 0, ms, n).                                            */
 int h2o_set_profiling(h2o_t h, int on);
@@ -165,8 +167,9 @@ int h2o_select(const float* scores, const int32_t* positions, int n_heads, int64
  *   device pointers of `dtype`;
  *   colsum [B, Hkv, M + S] float32 (device): colsum[.., c] for c < M is slot
  *   c's summed weight (0 for c >= n_valid), colsum[.., M + j] chunk key j's.
- * Limit: B * Hq * ceil(S / T) * (M + S) <= 4 * 2^20, with T = 128 (bf16, the
- * tensor-core kernel) or 64 (float32); larger problems return H2O_ESHAPE.
+ * Limit: B * Hq * ceil(S / T) * W <= 4 * 2^20, with W = M + S rounded up to
+ * a multiple of 4 and T = 128 (bf16, the tensor-core kernel) or 64 (float32);
+ * larger problems return H2O_ESHAPE.
  * Set-up: the first call on a device looks up the device address of the
  * scratch array with that device current; make that first call before any
  * stream capture on the device.

@@ -229,6 +229,46 @@ def test_host_buffers_match_device_buffers(h2o):
     b.close()
 
 
+@pytest.mark.parametrize("base,kw,T", [
+    (0, {}, None),
+    (0, {"dtype": torch.bfloat16, "d": 128, "M": 301, "R": 45, "P": 203, "S": 37}, 203 + 6 * 37 + 11),
+    (1, {}, 2048 + 3 * 1024),
+])
+def test_fused_tail_matches_split_kernels(h2o, monkeypatch, base, kw, T):
+    """The fused cluster tail and the three separate kernels sum the partial
+    rows in the same order, so outputs, state and cache agree bit for bit."""
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    cfg = _cfg(base, **kw)
+    T = cfg.T if T is None else T
+    Q, K, V = gen_batch(cfg, 0, device="cuda", T=T)
+    bounds = [(a, b) for a, b in cfg.bounds() if a < T]
+    bounds[-1] = (bounds[-1][0], min(bounds[-1][1], T))
+    chunks = split_chunks(Q, K, V, bounds)
+    fused = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    monkeypatch.setenv("H2O_SPLIT_TAIL", "1")
+    split = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    for ci, (q, k, v) in enumerate(chunks):
+        if ci == 0:
+            monkeypatch.delenv("H2O_SPLIT_TAIL")
+            of = fused.prefill(q, k, v)
+            monkeypatch.setenv("H2O_SPLIT_TAIL", "1")
+            os_ = split.prefill(q, k, v)
+        else:
+            monkeypatch.delenv("H2O_SPLIT_TAIL")
+            of = fused.step(q, k, v)
+            monkeypatch.setenv("H2O_SPLIT_TAIL", "1")
+            os_ = split.step(q, k, v)
+        assert fused.info()["launches"] == 2
+        assert split.info()["launches"] == 4
+        assert torch.equal(of, os_), f"chunk {ci}: outputs differ"
+        for x, y in zip(fused.read_state(), split.read_state()):
+            assert torch.equal(x, y), f"chunk {ci}: state differs"
+    for x, y in zip(fused.read_kv(), split.read_kv()):
+        assert torch.equal(x, y)
+    fused.close()
+    split.close()
+
+
 def test_standalone_select_with_ties(h2o):
     rng = np.random.default_rng(11)
     for trial in range(12):
