@@ -17,6 +17,15 @@
 //            sum, no cross-thread reduction) and writes them to shared memory
 //            as P^T; then O^T += V^T P^T (M = 128 = d, N = 256 queries), both
 //            operands MN-major.
+// Split keys: a unit of work (two heads' 128 rows) may be shared by a cluster
+// of kc CTAs, each taking a contiguous run of its 256-key pairs.  After sweep 1
+// every CTA publishes its rows' (max, sum) in shared memory, and each CTA
+// combines all of them in rank order into the same log-sum-exp (distributed
+// shared memory, remote mbarrier arrivals); after sweep 2 the partial O of
+// every CTA is staged in shared memory and rank q adds, in rank order, the
+// partials of its 256 / kc rows.  Column sums need no exchange: every key
+// belongs to one CTA.  Small chunks (S = 128: two-heads units are few) and
+// grids that would leave a partial last wave use kc > 1.
 // Exact probabilities mean O needs no rescaling.  Every MMA has N = 256: with
 // both operands in shared memory that is what keeps the tensor core near its
 // peak (N = 128 runs at about 70% of it).  Each (head, key) column sum of the
@@ -59,10 +68,16 @@ constexpr uint32_t kOffP = kOffR + NS2 * kTile;
 constexpr uint32_t kRBytes = NS2 * kTile + 2 * kTile;   // 160 KB
 constexpr uint32_t kOffLse = kOffR + kRBytes;           // negated base-2 lse, [2][128]
 constexpr uint32_t kOffBar = kOffLse + 2 * BM * 4;
-constexpr int kNumBars = 24;
+constexpr int kNumBars = 26;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffCs = kOffMisc + 16;             // head B's column sums of a tile, [128]
 constexpr uint32_t kSmemUsed = kOffCs + BN * 4;
+// cluster exchange of sweep-1 (max, sum) pairs, [2][128] float2: the part of
+// R that neither the sweep-1 slots nor the sweep-2 ring use, and that P^T
+// first overwrites only after every CTA of the cluster has read it
+constexpr uint32_t kOffX = kOffR + 2 * kSlot1;
+static_assert(kOffX >= kOffP && kOffX + 2 * BM * 8 <= kOffR + kRBytes, "exchange inside P^T's tail");
+constexpr int kMaxSplit = 8;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // slack for 1024-byte alignment
 static_assert(2 * kSlot1 <= kRBytes, "sweep-1 slots fit in R");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -73,14 +88,15 @@ enum { B_Q = 0, B_R1_FULL = 1, B_R1_EMPTY = 3, B_R2_FULL = 5, B_R2_EMPTY = B_R2_
        B_S_FULL = B_R2_EMPTY + NS2, B_S_EMPTY = B_S_FULL + 2, B_ST_FULL = B_S_EMPTY + 2,
        B_ST_EMPTY = B_ST_FULL + 1, B_P_FULL = B_ST_EMPTY + 1, B_P_EMPTY = B_P_FULL + 1,
        B_O_FULL = B_P_EMPTY + 1, B_DRAIN = B_O_FULL + 1, B_CS_FULL = B_DRAIN + 1,
-       B_CS_EMPTY = B_CS_FULL + 1 };
-static_assert(B_CS_EMPTY < kNumBars, "barrier count");
+       B_CS_EMPTY = B_CS_FULL + 1, B_X_READY = B_CS_EMPTY + 1, B_X_READ = B_X_READY + 1 };
+static_assert(B_X_READ < kNumBars, "barrier count");
 
 struct Params {
   float* partials;
   int* err;
   void* out;
   int B, Hq, Hkv, G, n_pg, n_rt;
+  int kc;                          // CTAs (a cluster) per unit of work
   int64_t S, M, n_valid, stride;   // stride: floats between partial rows
   float scale_log2;   // (1/sqrt(d)) * log2(e)
 };
@@ -174,9 +190,12 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- work unit: (b, h) major, then row tiles from the last (heaviest), then head pairs
+  const int kc = p.kc;
+  const int rank = (int)(blockIdx.x % (unsigned)kc);        // rank in the cluster
+  const int unit = (int)(blockIdx.x / (unsigned)kc);
   const int per_bh = p.n_pg * p.n_rt;
-  const int bh = blockIdx.x / per_bh;
-  const int k_in = blockIdx.x - bh * per_bh;
+  const int bh = unit / per_bh;
+  const int k_in = unit - bh * per_bh;
   const int rt = p.n_rt - 1 - k_in / p.n_pg;
   const int pg = k_in % p.n_pg;
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
@@ -186,8 +205,15 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int nct = (int)((p.n_valid + BN - 1) / BN);         // cache tiles
   const int64_t chunk_hi = (i0 + BM < p.S) ? i0 + BM : p.S;   // chunk keys < chunk_hi are visible
   const int nch = (int)((chunk_hi + BN - 1) / BN);
-  const int n = nct + nch;                                    // 128-key tiles
-  const int n1 = (n + 1) >> 1;                                // sweep-1 256-key tiles
+  const int n_all = nct + nch;                                // the unit's 128-key tiles
+  const int n1_all = (n_all + 1) >> 1;                        // and its 256-key pairs
+  // this CTA's pairs [pr0, pr1), i.e. tiles [t_lo, t_hi); the launch keeps
+  // kc <= n1_all, so no CTA is left without keys
+  const int pr0 = (int)((int64_t)rank * n1_all / kc), pr1 = (int)((int64_t)(rank + 1) * n1_all / kc);
+  const int t_lo = 2 * pr0;
+  const int t_hi = 2 * pr1 < n_all ? 2 * pr1 : n_all;
+  const int n = t_hi - t_lo;                                  // local 128-key tiles
+  const int n1 = pr1 - pr0;                                   // local 256-key tiles
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
@@ -195,6 +221,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (i == B_S_EMPTY || i == B_S_EMPTY + 1) cnt = 128;   // one warpgroup
       if (i == B_ST_EMPTY || i == B_P_FULL) cnt = 256;        // both warpgroups
       if (i == B_CS_FULL || i == B_CS_EMPTY) cnt = 128;       // one warpgroup
+      if (i == B_X_READY || i == B_X_READ) cnt = (uint32_t)kc;  // one arrival per CTA
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -206,19 +233,21 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
   tc_fence_before();
   __syncthreads();
+  if (kc > 1) cluster_sync_all();   // every CTA's barriers exist before remote arrivals
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // the cache and the partial rows may still be in use by the previous kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // tile t (128 keys): tensor map and row offset
+  // local tile t (128 keys), i.e. the unit's tile t_lo + t: tensor map and row offset
   auto tile_src = [&](int t, bool v, const CUtensorMap*& m, int& y) {
-    if (t < nct) {
+    const int tg = t_lo + t;
+    if (tg < nct) {
       m = v ? &tm_vc : &tm_kc;
-      y = t * BN;
-    } else if (t < n) {
+      y = tg * BN;
+    } else if (tg < t_hi) {
       m = v ? &tm_v : &tm_k;
-      y = (t - nct) * BN;
+      y = (tg - nct) * BN;
     } else {  // past the last tile: a box beyond the chunk's rows reads zeros
       m = v ? &tm_v : &tm_k;
       y = (int)p.S;
@@ -395,9 +424,10 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float m = -INFINITY, l = 0.f;
     const uint32_t s_tmem = lane_base + (uint32_t)w * 256u;
     auto nvis_of = [&](int t, int half64) -> int {
-      if (t >= n) return 0;
-      const bool cache = t < nct;
-      const int64_t key0 = (cache ? (int64_t)t * BN : (int64_t)(t - nct) * BN) + half64 * 64;
+      const int tg = t_lo + t;
+      if (tg >= t_hi) return 0;
+      const bool cache = tg < nct;
+      const int64_t key0 = (cache ? (int64_t)tg * BN : (int64_t)(tg - nct) * BN) + half64 * 64;
       const int64_t lim = cache ? nv : row_lim;
       return (int)(lim - key0 > 64 ? 64 : (lim - key0 < 0 ? 0 : lim - key0));
     };
@@ -429,7 +459,42 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       __syncwarp();
     }
     // negated base-2 log-sum-exp of each row; -inf zeroes rows past S and a missing head B
-    nlse[w * BM + r] = (head_ok && row_i < S && l > 0.f) ? -(m + lg2(l)) : -INFINITY;
+    if (kc == 1) {
+      nlse[w * BM + r] = (head_ok && row_i < S && l > 0.f) ? -(m + lg2(l)) : -INFINITY;
+    } else {
+      // publish this CTA's (m, l); once every CTA has, combine them in rank order
+      const uint32_t x_own = base + kOffX + (uint32_t)(w * BM + r) * 8u;
+      *reinterpret_cast<float2*>(sbase + kOffX + (w * BM + r) * 8) = make_float2(m, l);
+      named_bar_sync(3, 256);
+      if (threadIdx.x == 64) {
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        for (int q = 0; q < kc; ++q) mbar_arrive_remote(cluster_map(bar(B_X_READY), (uint32_t)q));
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_X_READY), 0, abort_flag, p.err, kWaitLimitNs,
+                                                   kErrTimeout));
+      float mq[kMaxSplit], lq[kMaxSplit];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < kMaxSplit; ++q) {
+        mq[q] = -INFINITY;
+        lq[q] = 0.f;
+        if (ok && q < kc) {
+          const float2 x = ld_cluster_f2(cluster_map(x_own, (uint32_t)q));
+          mq[q] = x.x;
+          lq[q] = x.y;
+          if (x.y > 0.f) mx = fmaxf(mx, x.x);
+        }
+      }
+      float lsum = 0.f;
+#pragma unroll
+      for (int q = 0; q < kMaxSplit; ++q)
+        if (lq[q] > 0.f) lsum += lq[q] * ex2(mq[q] - mx);
+      nlse[w * BM + r] = (head_ok && row_i < S && lsum > 0.f) ? -(mx + lg2(lsum)) : -INFINITY;
+      // every CTA's exchange area is overwritten by P^T only after all have read it
+      named_bar_sync(3, 256);
+      if (threadIdx.x == 64)
+        for (int q = 0; q < kc; ++q) mbar_arrive_remote(cluster_map(bar(B_X_READ), (uint32_t)q));
+    }
     named_bar_sync(1 + w, 128);
 
     // ----- sweep 2: thread = key (lane r of S^T), the 128 query columns of head w
@@ -457,8 +522,9 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_arrive(bar(B_CS_EMPTY));
         if (prev_col >= 0) part[prev_col] = prev_cs + other;
       }
-      const bool cache = j < nct;
-      const int64_t key = cache ? (int64_t)j * BN + r : (int64_t)(j - nct) * BN + r;
+      const int jg = t_lo + j;
+      const bool cache = jg < nct;
+      const int64_t key = cache ? (int64_t)jg * BN + r : (int64_t)(jg - nct) * BN + r;
       const bool key_ok = cache ? key < nv : key < S;
       // chunk key `key` is seen by query columns q with i0 + q >= key
       const int qmin = cache ? 0 : (int)(key - i0 > 0 ? key - i0 : 0);
@@ -480,6 +546,11 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(B_ST_EMPTY));
+        if (kc > 1 && j == 0) {   // the cluster is done with the exchange area
+          ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_X_READ), 0, abort_flag, p.err,
+                                                       kWaitLimitNs, kErrTimeout));
+          if (!ok) break;
+        }
         // this warpgroup's P^T half of the previous tile has been read by its O^T MMA:
         // store the first 64 queries now, the second half's exponentials overlap it
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
@@ -514,7 +585,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // ----- epilogue: O^T (lane = d, columns = queries) -> out rows via shared memory
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), 0, abort_flag, p.err,
                                                    kWaitLimitNs, kErrTimeout));
-    if (ok) {
+    if (ok && kc == 1) {
       tc_fence_after();
       // every MMA has completed: R is free; head w's [128 queries x 128 d] goes to R + w * 32 KB
       __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sbase + kOffR + (uint32_t)w * kTile);
@@ -536,7 +607,55 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
         for (int k = 0; k < D * 2 / 16; ++k) dst[k] = src[k];
       }
+    } else if (ok) {
+      tc_fence_after();
+      // this CTA's partial O, fp32 [256 queries][128 d], to R (free: every MMA has completed)
+      float* stage = reinterpret_cast<float*>(sbase + kOffR);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + 256u + (uint32_t)w * 128u + ch * 32, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) stage[(w * BM + ch * 32 + k) * D + r] = __uint_as_float(o[k]);
+      }
     }
+  }
+
+  if (kc > 1) {
+    // every CTA has staged its partial O; rank q sums, in rank order, the rows
+    // [q * 256 / kc, (q + 1) * 256 / kc) of all of them and writes them out
+    __syncthreads();
+    cluster_sync_all();
+    if (warp >= 2 && p.out != nullptr) {
+      const int t = threadIdx.x - 64;                 // 0..255
+      const int rows = 2 * BM / kc;
+      const uint32_t stage0 = base + kOffR;
+      for (int it = t; it < rows * (D / 8); it += 256) {
+        const int q = rank * rows + it / (D / 8);     // query 0..255: head q / 128, row q % 128
+        const int d0 = (it % (D / 8)) * 8;
+        const uint32_t off = stage0 + (uint32_t)(q * D + d0) * 4u;
+        float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+        for (int src = 0; src < kc; ++src) {
+          const float4 a = ld_cluster_f4(cluster_map(off, (uint32_t)src));
+          const float4 c4 = ld_cluster_f4(cluster_map(off + 16u, (uint32_t)src));
+          lo.x += a.x; lo.y += a.y; lo.z += a.z; lo.w += a.w;
+          hi.x += c4.x; hi.y += c4.y; hi.z += c4.z; hi.w += c4.w;
+        }
+        const int wq = q / BM;
+        const int64_t qi = i0 + (q % BM);
+        if ((wq == 0 || has_b) && qi < p.S) {
+          const int g = h * p.G + gl_a + wq;
+          uint4 v;
+          v.x = pack_bf16(lo.x, lo.y);
+          v.y = pack_bf16(lo.z, lo.w);
+          v.z = pack_bf16(hi.x, hi.y);
+          v.w = pack_bf16(hi.z, hi.w);
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (((int64_t)b * p.Hq + g) * p.S + qi) * D + d0) = v;
+        }
+      }
+    }
+    cluster_sync_all();   // no CTA leaves while another reads its stage
   }
 
   tc_fence_before();
@@ -575,6 +694,65 @@ cudaError_t make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t z) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Clusters of kc CTAs that fit on the device at once (1 CTA per SM), per device.
+int active_clusters(int kc) {
+  static std::mutex mu;
+  static int cache[64][kMaxSplit + 1] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 0;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev][kc] == 0) {
+    int n = 0;
+    if (kc == 1) {
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    } else {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)kc);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = (unsigned)kc;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, attn_umma_kernel, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    cache[dev][kc] = n > 0 ? n : -1;
+  }
+  return cache[dev][kc] > 0 ? cache[dev][kc] : 0;
+}
+
+// CTAs per unit of work.  `forced` > 0 asks for that split (capped by what the
+// sizes allow); otherwise the split is the one whose waves of clusters take the
+// least time, ceil(units / active clusters) / kc, needing a 10% gain over no
+// split to pay for the exchanges.  Every CTA keeps at least one 256-key pair.
+int split_for(int64_t units, int min_pairs, int forced) {
+  int best_kc = 1;
+  const int sm = active_clusters(1);
+  double best = sm > 0 ? (double)((units + sm - 1) / sm) : 1.0;
+  for (int kc = 2; kc <= kMaxSplit; kc *= 2) {
+    if (kc > min_pairs) break;
+    const int nclu = active_clusters(kc);
+    if (nclu < 1) continue;
+    if (forced > 0) {
+      if (kc <= forced) best_kc = kc;
+      continue;
+    }
+    const double t = (double)((units + nclu - 1) / nclu) / kc;
+    if (t < 0.9 * best) {
+      best = t;
+      best_kc = kc;
+    }
+  }
+  return best_kc;
+}
+
 }  // namespace
 
 bool attn_umma_supported(int dtype, int d) { return dtype == kBF16 && d == D; }
@@ -609,17 +787,23 @@ cudaError_t launch_attn_umma(const AttnArgs& a, bool pdl, cudaStream_t st) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   e = cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int64_t grid = BHkv * p.n_pg * p.n_rt;
+  const int64_t units = BHkv * p.n_pg * p.n_rt;
+  const int nct = (int)((a.n_valid + BN - 1) / BN);
+  p.kc = split_for(units, (nct + 2) / 2, a.split);   // row tile 0 sees nct + 1 tiles
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
+  cfg.gridDim = dim3((unsigned)(units * p.kc));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = (unsigned)p.kc;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.kc > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, attn_umma_kernel, mq, mk, mv, mkc, mvc, p);
 }
 

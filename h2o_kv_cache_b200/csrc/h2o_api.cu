@@ -133,6 +133,13 @@ bool split_tail() {
   return s && s[0] == '1';
 }
 
+// H2O_ATTN_SPLIT=k asks the tensor-core attention kernel to split each unit of
+// work over k CTAs (a cluster; capped by the sizes); unset, it chooses.
+int attn_split() {
+  const char* s = getenv("H2O_ATTN_SPLIT");
+  return s ? atoi(s) : 0;
+}
+
 bool sync_check_enabled() {
   const char* s = getenv("H2O_SYNC_CHECK");
   return s && s[0] == '1';
@@ -240,6 +247,7 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   a.M = h->M;
   a.n_valid = h->n_valid;
   a.part_stride = stride;
+  a.split = attn_split();
   a.scale = (float)(1.0 / std::sqrt((double)h->d));
   if (fault_injected("launch")) return fail(h, H2O_ECUDA, "injected launch failure");
   cudaError_t e = h->use_umma ? h2o::launch_attn_umma(a, true, st)

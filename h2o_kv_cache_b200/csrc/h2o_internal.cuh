@@ -49,6 +49,7 @@ struct AttnArgs {
   int B, Hq, Hkv, d;
   int64_t S, M, n_valid, part_stride;
   float scale;        // 1/sqrt(d)
+  int split = 0;      // tensor-core kernel: CTAs per unit of work (0 = chosen by occupancy)
 };
 
 // Row-tile height of each attention implementation (sets the partials layout).

@@ -154,6 +154,30 @@ def test_window_just_below_capacity(h2o):
     run_stream(h2o, cfg)
 
 
+@pytest.mark.parametrize("split", ["2", "4", "8"])
+def test_keys_split_across_a_cluster(h2o, monkeypatch, split):
+    # each unit's keys shared by `split` CTAs: exchanged row statistics and summed partial O
+    monkeypatch.setenv("H2O_ATTN_SPLIT", split)
+    cfg = _cfg(1)
+    s = run_stream(h2o, cfg, heads=[(0, 0), (0, 5)], T=cfg.P + 2 * cfg.S)
+    assert s["chunks"] == 3
+
+
+def test_split_with_odd_tile_counts(h2o, monkeypatch):
+    # 8 cache tiles + 1-2 chunk tiles per unit: the last CTA of a cluster gets an odd tile
+    monkeypatch.setenv("H2O_ATTN_SPLIT", "4")
+    cfg = _cfg(0, name="split-odd", B=1, Hq=6, Hkv=2, d=128, M=1000, R=90, T=1000 + 4 * 200 + 77,
+               P=1000, S=200, dtype=torch.bfloat16, planted=0.02)
+    run_stream(h2o, cfg)
+
+
+def test_small_chunks_s128(h2o):
+    # S = 128: 16 units for 148 SMs, so the kernel splits each unit's keys
+    cfg = _cfg(1, name="m2k-s128", S=128)
+    s = run_stream(h2o, cfg, T=cfg.P + 6 * 128)
+    assert s["chunks"] == 7
+
+
 # --------------------------------------------------------------------------------------
 # The benchmark workloads at full size
 # --------------------------------------------------------------------------------------
