@@ -88,8 +88,9 @@ enum { B_Q = 0, B_R1_FULL = 1, B_R1_EMPTY = 3, B_R2_FULL = 5, B_R2_EMPTY = B_R2_
        B_S_FULL = B_R2_EMPTY + NS2, B_S_EMPTY = B_S_FULL + 2, B_ST_FULL = B_S_EMPTY + 2,
        B_ST_EMPTY = B_ST_FULL + 1, B_P_FULL = B_ST_EMPTY + 1, B_P_EMPTY = B_P_FULL + 1,
        B_O_FULL = B_P_EMPTY + 1, B_DRAIN = B_O_FULL + 1, B_CS_FULL = B_DRAIN + 1,
-       B_CS_EMPTY = B_CS_FULL + 1, B_X_READY = B_CS_EMPTY + 1, B_X_READ = B_X_READY + 1 };
-static_assert(B_X_READ < kNumBars, "barrier count");
+       B_CS_EMPTY = B_CS_FULL + 1, B_X_READY = B_CS_EMPTY + 1, B_X_READ = B_X_READY + 1,
+       B_NEVER = B_X_READ + 1 };   // test hook: nothing ever arrives on it
+static_assert(B_NEVER < kNumBars, "barrier count");
 
 struct Params {
   float* partials;
@@ -97,6 +98,7 @@ struct Params {
   void* out;
   int B, Hq, Hkv, G, n_pg, n_rt;
   int kc;                          // CTAs (a cluster) per unit of work
+  int inject_timeout;              // test hook: make one wait run out
   int64_t S, M, n_valid, stride;   // stride: floats between partial rows
   float scale_log2;   // (1/sqrt(d)) * log2(e)
 };
@@ -270,6 +272,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tma_load_3d(base + kOffQ + at * 2 * kAtom + hw * kAtom, &tm_q, bar(B_Q), at * 64, (int)i0,
                       zq + hw);
       bool ok = true;
+      int issued1 = 0;                               // sweep-1 tiles whose loads were issued
       // sweep 1: 256-key K tiles into two 64 KB slots
       for (int u = 0; ok && u < n1; ++u) {
         const int s = u & 1;
@@ -285,6 +288,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int at = 0; at < 2; ++at)
             tma_load_3d(dst + at * 2 * kAtom + half * kAtom, m, bar(B_R1_FULL + s), at * 64, y, bh);
         }
+        issued1 = u + 1;
       }
       // sweep 2 reuses R: wait until every sweep-1 slot has been read
       for (int s = 0; ok && s < 2; ++s) {
@@ -314,10 +318,13 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tma_load_3d(dst + kAtom, m, bar(B_R2_FULL + slot), 64, y, bh);
         issued = pos + 1;
       }
-      // drain: the last load of each slot has landed before the CTA may exit
+      // drain, also after an abort: every load issued has landed before the CTA may exit
+      mbar_drain(bar(B_Q), 0, p.err, kWaitLimitNs, kErrTimeout);
+      for (int u = issued1 - 2 < 0 ? 0 : issued1 - 2; u < issued1; ++u)
+        mbar_drain(bar(B_R1_FULL + (u & 1)), (uint32_t)(u >> 1) & 1u, p.err, kWaitLimitNs, kErrTimeout);
       for (int pos = issued - NS2 < 0 ? 0 : issued - NS2; pos < issued; ++pos)
-        mbar_wait(bar(B_R2_FULL + pos % NS2), (uint32_t)(pos / NS2) & 1u, abort_flag, p.err,
-                  kWaitLimitNs, kErrTimeout);
+        mbar_drain(bar(B_R2_FULL + pos % NS2), (uint32_t)(pos / NS2) & 1u, p.err, kWaitLimitNs,
+                   kErrTimeout);
     }
   } else if (warp == 1) {
     // =========================================================== MMA issuer
@@ -400,9 +407,9 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       if (ok) ok = issue_ot(n - 1);
       umma_commit(bar(B_O_FULL));
-      // every MMA issued has completed before TMEM is released
+      // every MMA issued has completed before TMEM is released, also after an abort
       umma_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, abort_flag, p.err, kWaitLimitNs, kErrTimeout);
+      mbar_drain(bar(B_DRAIN), 0, p.err, kWaitLimitNs, kErrTimeout);
     }
   } else {
     // =========================================================== softmax / epilogue
@@ -414,6 +421,11 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const float c = p.scale_log2;
     const bool head_ok = w == 0 || has_b;
     bool ok = true;
+    if (p.inject_timeout && w == 0) {
+      // test hook: a bounded wait on a barrier nothing completes runs out (1 ms);
+      // every role then leaves through its abort path and the step reports it
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_NEVER), 0, abort_flag, p.err, 1000000ull, kErrTimeout));
+    }
 
     // ----- sweep 1: thread = query row i0 + r of head w; running (max, sum).
     // The sum is kept against a reference max that is only raised when a
@@ -784,6 +796,7 @@ cudaError_t launch_attn_umma(const AttnArgs& a, bool pdl, cudaStream_t st) {
   p.M = a.M;
   p.n_valid = a.n_valid;
   p.stride = a.part_stride;
+  p.inject_timeout = a.inject_timeout;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   e = cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;

@@ -140,6 +140,14 @@ int attn_split() {
   return s ? atoi(s) : 0;
 }
 
+// H2O_INJECT_TIMEOUT=1 (test hook): in the tensor-core attention kernel one
+// softmax warpgroup waits on a barrier that nothing completes, with a 1 ms
+// limit; the step then fails with H2O_ETIMEOUT and the context stays usable.
+bool inject_timeout() {
+  const char* s = getenv("H2O_INJECT_TIMEOUT");
+  return s && s[0] == '1';
+}
+
 bool sync_check_enabled() {
   const char* s = getenv("H2O_SYNC_CHECK");
   return s && s[0] == '1';
@@ -248,6 +256,7 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   a.n_valid = h->n_valid;
   a.part_stride = stride;
   a.split = attn_split();
+  a.inject_timeout = inject_timeout() ? 1 : 0;
   a.scale = (float)(1.0 / std::sqrt((double)h->d));
   if (fault_injected("launch")) return fail(h, H2O_ECUDA, "injected launch failure");
   cudaError_t e = h->use_umma ? h2o::launch_attn_umma(a, true, st)

@@ -50,6 +50,7 @@ struct AttnArgs {
   int64_t S, M, n_valid, part_stride;
   float scale;        // 1/sqrt(d)
   int split = 0;      // tensor-core kernel: CTAs per unit of work (0 = chosen by occupancy)
+  int inject_timeout = 0;   // tensor-core kernel, test hook: one bounded wait runs out
 };
 
 // Row-tile height of each attention implementation (sets the partials layout).

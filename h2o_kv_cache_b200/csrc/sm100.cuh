@@ -131,6 +131,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// For copies and MMAs this CTA issued itself, which complete on their own:
+// waits for the phase even after another role has aborted (the CTA must not
+// free TMEM or exit with them in flight), for at most ~limit_ns.
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, int* err, uint64_t limit_ns,
+                                           int err_bit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0 && global_timer_ns() - t0 > limit_ns) {
+      atomicOr(err, err_bit);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 // 3-d tiled load of a box into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,

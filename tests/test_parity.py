@@ -232,6 +232,28 @@ def test_shape_error_leaves_state_intact(h2o):
     cache.close()
 
 
+def test_bounded_wait_timeout_is_reported_and_context_stays_usable(h2o, monkeypatch):
+    # a wait on a barrier that nothing completes runs out (1 ms); every role of the
+    # kernel leaves through its abort path, the step reports H2O_ETIMEOUT, and the
+    # device context keeps working
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    cfg = _cfg(0, dtype=torch.bfloat16, d=128)
+    Q, K, V = gen_batch(cfg, 0, device="cuda")
+    chunks = split_chunks(Q, K, V, cfg.bounds())
+    cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    cache.prefill(*chunks[0])
+    monkeypatch.setenv("H2O_INJECT_TIMEOUT", "1")
+    monkeypatch.setenv("H2O_SYNC_CHECK", "1")
+    with pytest.raises(h2o.H2OError) as ei:
+        cache.step(*chunks[1])
+    assert ei.value.status == -6, ei.value
+    cache.close()
+    monkeypatch.delenv("H2O_INJECT_TIMEOUT")
+    monkeypatch.delenv("H2O_SYNC_CHECK")
+    s = run_stream(h2o, cfg)
+    assert s["chunks"] == 5
+
+
 def test_host_buffers_match_device_buffers(h2o):
     from h2o_kv_cache_b200.workload import gen_batch, split_chunks
     cfg = _cfg(0, dtype=torch.bfloat16, d=128)
