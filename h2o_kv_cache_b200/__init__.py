@@ -114,6 +114,17 @@ class H2OCache:
                                          _stream_ptr(stream, dev)))
         return slots, scores, pos
 
+    def read_delta(self, stream=None):
+        """The last step's buffer delta: (slots [B,Hkv,S_last] int32, the slots filled in
+        chunk order; evicted_positions [B,Hkv,S_last] int32, what each held before, -1 if
+        it was empty).  Chunk token i's K/V went to slots[..., i]."""
+        dev = self.device
+        slots = torch.empty(self.B, self.Hkv, self.last_S, dtype=torch.int32, device=dev)
+        evicted = torch.empty(self.B, self.Hkv, self.last_S, dtype=torch.int32, device=dev)
+        with torch.cuda.device(dev):
+            self._chk(lib.h2o_read_delta(self._h, _ptr(slots), _ptr(evicted), _stream_ptr(stream, dev)))
+        return slots, evicted
+
     def read_kv(self, stream=None):
         shape = (self.B, self.Hkv, self.M, self.d)
         kc = torch.empty(shape, dtype=self.dtype, device=self.device)

@@ -25,6 +25,7 @@ SIGNATURES = {
     "h2o_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp]),
     "h2o_read_state": (_i32, [_vp, _vp, _vp, _vp, _vp]),
     "h2o_read_kv": (_i32, [_vp, _vp, _vp, _vp]),
+    "h2o_read_delta": (_i32, [_vp, _vp, _vp, _vp]),
     "h2o_info": (_i32, [_vp, ctypes.POINTER(_i64)]),
     "h2o_set_profiling": (_i32, [_vp, _i32]),
     "h2o_step_timings": (_i32, [_vp, _i32, ctypes.POINTER(ctypes.c_float), _i32]),

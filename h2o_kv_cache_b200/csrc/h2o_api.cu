@@ -49,7 +49,7 @@ struct h2o_ctx {
   // device error word: mapped pinned host memory, so kernels report into it
   // directly and no copy is enqueued per step; nonzero only after an error
   int* err = nullptr;
-  DevBuf partials, newscore, freed;
+  DevBuf partials, newscore, freed, evicted;
   // staging for host pointers
   DevBuf st_q, st_k, st_v, st_out;
   cudaEvent_t err_ev = nullptr;   // recorded after each step
@@ -234,6 +234,7 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   const size_t part_bytes = (size_t)BH * n_grp * n_rt * stride * sizeof(float);
   H2O_CUDA(h, ensure(h->partials, part_bytes), "scratch alloc");
   H2O_CUDA(h, ensure(h->freed, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
+  H2O_CUDA(h, ensure(h->evicted, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
 
   cudaEvent_t* evs = h->ev[h->prof_steps % h2o_ctx::kProfRing];
   if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[0], st), "event");
@@ -278,6 +279,7 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
     t.kc = static_cast<uint4*>(h->kc);
     t.vc = static_cast<uint4*>(h->vc);
     t.freed = static_cast<int32_t*>(h->freed.p);
+    t.evicted = static_cast<int32_t*>(h->evicted.p);
     t.err = h->err;
     t.M = h->M;
     t.S = S;
@@ -304,7 +306,8 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
     if (e != cudaSuccess) return cuda_fail(h, e, "select launch");
     e = h2o::launch_scatter(dk, dv, h->kc, h->vc, h->scores, h->pos,
                             static_cast<int32_t*>(h->freed.p), static_cast<float*>(h->newscore.p),
-                            BH, S, h->M, h->d, (int)es, h->t0, st);
+                            static_cast<int32_t*>(h->evicted.p), BH, S, h->M, h->d, (int)es, h->t0,
+                            st);
     if (e != cudaSuccess) return cuda_fail(h, e, "scatter launch");
     h->last_launches = 4;
   }
@@ -438,6 +441,22 @@ int h2o_read_state(h2o_t h, int32_t* slots, float* scores, int32_t* positions, v
   return check_device_error(h, false);
 }
 
+int h2o_read_delta(h2o_t h, int32_t* slots, int32_t* evicted_positions, void* stream) {
+  if (!h) return fail(nullptr, H2O_EINVAL, "h2o_read_delta: NULL handle");
+  if (!h->prefilled) return fail(h, H2O_ESTATE, "h2o_read_delta: called before h2o_prefill");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)h->B * h->Hkv * h->last_S * sizeof(int32_t);
+  if (slots) H2O_CUDA(h, cudaMemcpyAsync(slots, h->freed.p, bytes, cudaMemcpyDefault, st), "copy slots");
+  if (evicted_positions)
+    H2O_CUDA(h, cudaMemcpyAsync(evicted_positions, h->evicted.p, bytes, cudaMemcpyDefault, st),
+             "copy evicted positions");
+  if ((slots && !is_device_ptr(slots)) || (evicted_positions && !is_device_ptr(evicted_positions))) {
+    H2O_CUDA(h, cudaStreamSynchronize(st), "read_delta sync");
+    return check_device_error(h, true);
+  }
+  return check_device_error(h, false);
+}
+
 int h2o_read_kv(h2o_t h, void* k_cache, void* v_cache, void* stream) {
   if (!h) return fail(nullptr, H2O_EINVAL, "h2o_read_kv: NULL handle");
   if (!h->prefilled) return fail(h, H2O_ESTATE, "h2o_read_kv: called before h2o_prefill");
@@ -497,7 +516,8 @@ int h2o_destroy(h2o_t h) {
   cudaFree(h->scores);
   cudaFree(h->pos);
   if (h->err) cudaFreeHost(h->err);
-  for (DevBuf* b : {&h->partials, &h->newscore, &h->freed, &h->st_q, &h->st_k, &h->st_v, &h->st_out})
+  for (DevBuf* b : {&h->partials, &h->newscore, &h->freed, &h->evicted, &h->st_q, &h->st_k, &h->st_v,
+                    &h->st_out})
     cudaFree(b->p);
   if (h->err_ev) cudaEventDestroy(h->err_ev);
   for (auto& set : h->ev)

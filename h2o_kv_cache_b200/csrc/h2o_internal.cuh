@@ -77,10 +77,12 @@ cudaError_t launch_select(const float* scores, const int32_t* pos, int BH, int64
                           int64_t t0, int64_t R, int64_t need, int64_t n_valid, int64_t S,
                           int32_t* freed, int64_t freed_stride, int* err, cudaStream_t st);
 
-// Chunk token i -> slot freed[bh, i]: K and V rows, pos = t0 + i, score = newscore[bh, i].
+// Chunk token i -> slot freed[bh, i]: K and V rows, pos = t0 + i, score = newscore[bh, i];
+// evicted[bh, i] = the position the slot held before (-1 if it was empty).
 cudaError_t launch_scatter(const void* k, const void* v, void* kc, void* vc, float* scores,
-                           int32_t* pos, const int32_t* freed, const float* newscore, int BH,
-                           int64_t S, int64_t M, int d, int esize, int64_t t0, cudaStream_t st);
+                           int32_t* pos, const int32_t* freed, const float* newscore,
+                           int32_t* evicted, int BH, int64_t S, int64_t M, int d, int esize,
+                           int64_t t0, cudaStream_t st);
 
 // The three steps above as one launch: one thread-block cluster per (b, KV
 // head).  freed[bh, 0..S) gets the same list launch_select writes.
@@ -93,6 +95,7 @@ struct TailArgs {
   uint4* kc;               // cache keys [BH, M, row_vecs]
   uint4* vc;               // cache values [BH, M, row_vecs]
   int32_t* freed;          // [BH, S]
+  int32_t* evicted;        // [BH, S]: position each freed slot held before (-1: was empty)
   int* err;
   int64_t M, S, n_valid, t0, R, need, stride;
   int n_grp, n_rt, row_tile, row_vecs;

@@ -190,7 +190,8 @@ __global__ void scatter_kernel(const uint4* __restrict__ k, const uint4* __restr
                                uint4* __restrict__ kc, uint4* __restrict__ vc,
                                float* __restrict__ scores, int32_t* __restrict__ pos,
                                const int32_t* __restrict__ freed, const float* __restrict__ newscore,
-                               int BH, int64_t S, int64_t M, int row_vecs, int64_t t0) {
+                               int32_t* __restrict__ evicted, int BH, int64_t S, int64_t M,
+                               int row_vecs, int64_t t0) {
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= (int64_t)BH * S) return;
@@ -204,6 +205,7 @@ __global__ void scatter_kernel(const uint4* __restrict__ k, const uint4* __restr
     vc[dst + c] = v[src + c];
   }
   if (lane == 0) {
+    evicted[bh * S + i] = pos[bh * M + slot];
     pos[bh * M + slot] = (int32_t)(t0 + i);
     scores[bh * M + slot] = newscore[bh * S + i];
   }
@@ -230,15 +232,16 @@ cudaError_t launch_select(const float* scores, const int32_t* pos, int BH, int64
 }
 
 cudaError_t launch_scatter(const void* k, const void* v, void* kc, void* vc, float* scores,
-                           int32_t* pos, const int32_t* freed, const float* newscore, int BH,
-                           int64_t S, int64_t M, int d, int esize, int64_t t0, cudaStream_t st) {
+                           int32_t* pos, const int32_t* freed, const float* newscore,
+                           int32_t* evicted, int BH, int64_t S, int64_t M, int d, int esize,
+                           int64_t t0, cudaStream_t st) {
   const int row_vecs = d * esize / 16;
   const int warps = 8;
   const int64_t rows = (int64_t)BH * S;
   const unsigned blocks = (unsigned)((rows + warps - 1) / warps);
   scatter_kernel<<<blocks, warps * 32, 0, st>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(kc),
-      static_cast<uint4*>(vc), scores, pos, freed, newscore, BH, S, M, row_vecs, t0);
+      static_cast<uint4*>(vc), scores, pos, freed, newscore, evicted, BH, S, M, row_vecs, t0);
   return cudaGetLastError();
 }
 

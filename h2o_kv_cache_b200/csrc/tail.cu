@@ -21,7 +21,8 @@
 //   3. ordered compaction: per-CTA counts are exchanged through rank 0, and
 //      each CTA writes its evicted slots at its offset, ascending;
 //   4. scatter of the CTA's chunk rows into the freed slots (the rows are read
-//      at the start, so only the stores remain here).
+//      at the start, so only the stores remain here), recording the position
+//      each slot held before: with the freed list, the chunk's buffer delta.
 #include <cstdint>
 
 #include "h2o_internal.cuh"
@@ -375,6 +376,7 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
   if (!sel_ok) return;
   auto finish_row = [&](int64_t i, int32_t slot) {
     if (lane == 0) {
+      p.evicted[bh * S + i] = p.pos[bh * M + slot];   // the delta record of this chunk row
       p.pos[bh * M + slot] = (int32_t)(p.t0 + i);
       p.scores[bh * M + slot] = ns[i - lo_s];
     }

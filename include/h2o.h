@@ -107,6 +107,19 @@ int h2o_step(h2o_t h, const void* q, const void* k, const void* v, void* out,
  * Errors: H2O_ESTATE before prefill.                                          */
 int h2o_read_state(h2o_t h, int32_t* slots, float* scores, int32_t* positions, void* stream);
 
+/* The last step's buffer delta ("Learning how to Forget: Fine-tuning for
+ * Long-Context Sparse Attention", Figure 1(c): per chunk, the slots written
+ * and the tokens they received), each pointer may be NULL to skip it:
+ *   slots              [B, Hkv, S_last] int32: the slots the step filled,
+ *                      ascending (as h2o_read_state returns them); chunk
+ *                      token i (its K/V rows are the step's own inputs) went
+ *                      to slots[.., i]
+ *   evicted_positions  [B, Hkv, S_last] int32: the token position slots[.., i]
+ *                      held before the step, -1 if it was empty.
+ * Together with the chunk's K/V these rebuild each step's cache from the
+ * previous one.  Errors: H2O_ESTATE before prefill.                           */
+int h2o_read_delta(h2o_t h, int32_t* slots, int32_t* evicted_positions, void* stream);
+
 /* Copy the cache contents out: k_cache, v_cache [B, Hkv, M, d] of the handle's
  * dtype (NULL skips).  Rows of empty slots are zero.                          */
 int h2o_read_kv(h2o_t h, void* k_cache, void* v_cache, void* stream);

@@ -70,6 +70,8 @@ def run_stream(h2o, cfg, heads=None, layer=0, T=None, oracle_chunks=None, kv_che
         if not follow:
             continue
         slots, scores, pos = (x.cpu().numpy() for x in cache.read_state())
+        d_slots, d_evicted = (x.cpu().numpy() for x in cache.read_delta())
+        assert np.array_equal(d_slots, slots)
         out64 = to64(out)
         qn = to64(q)
         kn_, vn_ = to64(k), to64(v)
@@ -85,6 +87,9 @@ def run_stream(h2o, cfg, heads=None, layer=0, T=None, oracle_chunks=None, kv_che
             status = check_evictions(st, slots[b, h], where)
             if status == "exact":
                 assert np.array_equal(pos[b, h], st.pos), f"{where}: slot -> position map differs"
+                # the buffer delta: each filled slot's previous token (-1: it was empty)
+                assert np.array_equal(d_evicted[b, h], pos_before[(b, h)][slots[b, h]]), \
+                    f"{where}: evicted positions differ"
                 summary["score_rel"] = max(summary["score_rel"],
                                            check_scores(scores[b, h], st.score, st.pos >= 0, where))
             else:
@@ -307,7 +312,7 @@ def test_fused_tail_matches_split_kernels(h2o, monkeypatch, base, kw, T):
         assert fused.info()["launches"] == 2
         assert split.info()["launches"] == 4
         assert torch.equal(of, os_), f"chunk {ci}: outputs differ"
-        for x, y in zip(fused.read_state(), split.read_state()):
+        for x, y in zip(fused.read_state() + fused.read_delta(), split.read_state() + split.read_delta()):
             assert torch.equal(x, y), f"chunk {ci}: state differs"
     for x, y in zip(fused.read_kv(), split.read_kv()):
         assert torch.equal(x, y)
