@@ -50,6 +50,9 @@ struct h2o_ctx {
   // directly and no copy is enqueued per step; nonzero only after an error
   int* err = nullptr;
   DevBuf partials, newscore, freed, evicted;
+  // stream-partitioned attention: per-piece row statistics, partial O, unit counters
+  DevBuf ws_ml, ws_o, ws_count;
+  int n_sm = 0;
   // staging for host pointers
   DevBuf st_q, st_k, st_v, st_out;
   cudaEvent_t err_ev = nullptr;   // recorded after each step
@@ -138,6 +141,17 @@ bool split_tail() {
 int attn_split() {
   const char* s = getenv("H2O_ATTN_SPLIT");
   return s ? atoi(s) : 0;
+}
+
+// H2O_ATTN_MODE=fused / stream forces one of the two tensor-core attention
+// paths (one kernel with both sweeps / two kernels over equal runs of key
+// pairs); unset, the choice below is made per launch.
+int attn_mode() {
+  const char* s = getenv("H2O_ATTN_MODE");
+  if (!s) return 0;
+  if (strcmp(s, "fused") == 0) return 1;
+  if (strcmp(s, "stream") == 0) return 2;
+  return 0;
 }
 
 // H2O_INJECT_TIMEOUT=1 (test hook): in the tensor-core attention kernel one
@@ -260,8 +274,32 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   a.inject_timeout = inject_timeout() ? 1 : 0;
   a.scale = (float)(1.0 / std::sqrt((double)h->d));
   if (fault_injected("launch")) return fail(h, H2O_ECUDA, "injected launch failure");
-  cudaError_t e = h->use_umma ? h2o::launch_attn_umma(a, true, st)
-                               : h2o::launch_attn_simt(a, h->dtype, true, st);
+  cudaError_t e = cudaSuccess;
+  int launches = 1;
+  if (h->use_umma) {
+    if (h->n_sm == 0) H2O_CUDA(h, cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device),
+                               "device attribute");
+    const int mode = attn_mode();
+    h2o::StreamPlan pl;
+    bool stream = false;
+    // automatic: a balanced partition pays when the one-kernel grid would
+    // leave SMs idle (n_sm / 2 .. 2 n_sm units) and units are long enough
+    // (>= 24 pairs on average) for a piece boundary's Q reload and epilogue
+    if (mode != 1 && !a.inject_timeout && h2o::attn_stream_plan(a, h->n_sm, &pl))
+      stream = mode == 2 || (2 * pl.units >= h->n_sm && pl.units <= 2 * h->n_sm &&
+                             pl.total_pairs >= 24 * (int64_t)pl.units);
+    if (stream) {
+      H2O_CUDA(h, ensure(h->ws_ml, pl.ml_bytes), "scratch alloc");
+      if (pl.o_bytes) H2O_CUDA(h, ensure(h->ws_o, pl.o_bytes), "scratch alloc");
+      H2O_CUDA(h, ensure(h->ws_count, pl.count_bytes), "scratch alloc");
+      e = h2o::launch_attn_stream(a, pl, h->ws_ml.p, h->ws_o.p, static_cast<int*>(h->ws_count.p), true, st);
+      launches = 2;
+    } else {
+      e = h2o::launch_attn_umma(a, true, st);
+    }
+  } else {
+    e = h2o::launch_attn_simt(a, h->dtype, true, st);
+  }
   if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
   if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[1], st), "event");
 
@@ -294,7 +332,7 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
     t.row_vecs = (int)(h->d * es / 16);
     e = h2o::launch_tail(t, BH, h->tail_cs, true, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "tail launch");
-    h->last_launches = 2;
+    h->last_launches = launches + 1;
   } else {
     H2O_CUDA(h, ensure(h->newscore, (size_t)BH * S * sizeof(float)), "scratch alloc");
     e = h2o::launch_score_reduce(static_cast<float*>(h->partials.p), h->scores,
@@ -309,7 +347,7 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
                             static_cast<int32_t*>(h->evicted.p), BH, S, h->M, h->d, (int)es, h->t0,
                             st);
     if (e != cudaSuccess) return cuda_fail(h, e, "scatter launch");
-    h->last_launches = 4;
+    h->last_launches = launches + 3;
   }
   if (h->prof) {
     H2O_CUDA(h, cudaEventRecord(evs[2], st), "event");
@@ -516,8 +554,8 @@ int h2o_destroy(h2o_t h) {
   cudaFree(h->scores);
   cudaFree(h->pos);
   if (h->err) cudaFreeHost(h->err);
-  for (DevBuf* b : {&h->partials, &h->newscore, &h->freed, &h->evicted, &h->st_q, &h->st_k, &h->st_v,
-                    &h->st_out})
+  for (DevBuf* b : {&h->partials, &h->newscore, &h->freed, &h->evicted, &h->ws_ml, &h->ws_o,
+                    &h->ws_count, &h->st_q, &h->st_k, &h->st_v, &h->st_out})
     cudaFree(b->p);
   if (h->err_ev) cudaEventDestroy(h->err_ev);
   for (auto& set : h->ev)

@@ -64,6 +64,19 @@ cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, bool pdl, cudaStream_
 cudaError_t launch_attn_umma(const AttnArgs& a, bool pdl, cudaStream_t st);
 bool attn_umma_supported(int dtype, int d);
 
+// Tensor-core attention as two persistent kernels over equal runs of all
+// units' 256-key pairs (attn_stream.cu).  attn_stream_plan() sizes the run
+// partition and the workspace for n_sm CTAs, or returns false when the
+// partition does not fit (then the one-kernel path runs).
+struct StreamPlan {
+  int n_cta = 0, maxp = 0, units = 0;
+  int64_t total_pairs = 0;
+  size_t ml_bytes = 0, o_bytes = 0, count_bytes = 0;   // workspace the caller provides
+};
+bool attn_stream_plan(const AttnArgs& a, int n_sm, StreamPlan* plan);
+cudaError_t launch_attn_stream(const AttnArgs& a, const StreamPlan& plan, void* ws_ml, void* ws_o,
+                               int* count, bool pdl, cudaStream_t st);
+
 // scores[b,h,c] += sum of partial column c (c < n_valid);
 // newscore[b,h,j] = sum of partial column M + j (j < S); n_grp partial groups.
 cudaError_t launch_score_reduce(const float* partials, float* scores, float* newscore, int BH,

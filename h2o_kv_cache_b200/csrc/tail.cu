@@ -374,9 +374,10 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
 
   // ---- 4. chunk row i -> slot fr[i]: K and V rows, pos = t0 + i, initial score
   if (!sel_ok) return;
-  auto finish_row = [&](int64_t i, int32_t slot) {
+  // old = the position the slot held: lane j read it with the slot of row j
+  auto finish_row = [&](int64_t i, int32_t slot, int32_t old) {
     if (lane == 0) {
-      p.evicted[bh * S + i] = p.pos[bh * M + slot];   // the delta record of this chunk row
+      p.evicted[bh * S + i] = old;                      // the delta record of this chunk row
       p.pos[bh * M + slot] = (int32_t)(p.t0 + i);
       p.scores[bh * M + slot] = ns[i - lo_s];
     }
@@ -385,18 +386,20 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
   if (pre_ok) {
     // lane k fetches the slot of the warp's k-th row
     const int32_t my_slot = lane < n_mine ? ld_relaxed(fr + lo_s + warp + (int64_t)lane * nwarps) : -1;
+    const int32_t my_old = (my_slot >= 0 && my_slot < M) ? p.pos[bh * M + my_slot] : -1;
 #pragma unroll
     for (int k = 0; k < kPre; ++k) {
       if (k < n_mine) {
         const int64_t i = lo_s + warp + (int64_t)k * nwarps;
         const int32_t slot = __shfl_sync(0xffffffffu, my_slot, k);
+        const int32_t old = __shfl_sync(0xffffffffu, my_old, k);
         if (slot < 0 || slot >= M) {
           if (lane == 0) atomicOr(p.err, kErrBounds);
         } else {
           const int64_t dst = (bh * M + slot) * rv;
           if (lane < rv) p.kc[dst + lane] = pre[k];
           else if (lane < vecs2) p.vc[dst + lane - rv] = pre[k];
-          finish_row(i, slot);
+          finish_row(i, slot, old);
         }
       }
     }
@@ -404,10 +407,12 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
   }
   for (int64_t k0 = k_from; k0 < n_mine; k0 += 32) {
     const int32_t my_slot = k0 + lane < n_mine ? ld_relaxed(fr + lo_s + warp + (k0 + lane) * nwarps) : -1;
+    const int32_t my_old = (my_slot >= 0 && my_slot < M) ? p.pos[bh * M + my_slot] : -1;
     const int kn = n_mine - k0 < 32 ? (int)(n_mine - k0) : 32;
     for (int jj = 0; jj < kn; ++jj) {
       const int64_t i = lo_s + warp + (k0 + jj) * nwarps;
       const int32_t slot = __shfl_sync(0xffffffffu, my_slot, jj);
+      const int32_t old = __shfl_sync(0xffffffffu, my_old, jj);
       if (slot < 0 || slot >= M) {
         if (lane == 0) atomicOr(p.err, kErrBounds);
         continue;
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
         if (c < rv) p.kc[dst + c] = __ldg(p.k + src + c);
         else p.vc[dst + c - rv] = __ldg(p.v + src + c - rv);
       }
-      finish_row(i, slot);
+      finish_row(i, slot, old);
     }
   }
 }

@@ -162,6 +162,7 @@ def test_window_just_below_capacity(h2o):
 @pytest.mark.parametrize("split", ["2", "4", "8"])
 def test_keys_split_across_a_cluster(h2o, monkeypatch, split):
     # each unit's keys shared by `split` CTAs: exchanged row statistics and summed partial O
+    monkeypatch.setenv("H2O_ATTN_MODE", "fused")
     monkeypatch.setenv("H2O_ATTN_SPLIT", split)
     cfg = _cfg(1)
     s = run_stream(h2o, cfg, heads=[(0, 0), (0, 5)], T=cfg.P + 2 * cfg.S)
@@ -170,10 +171,36 @@ def test_keys_split_across_a_cluster(h2o, monkeypatch, split):
 
 def test_split_with_odd_tile_counts(h2o, monkeypatch):
     # 8 cache tiles + 1-2 chunk tiles per unit: the last CTA of a cluster gets an odd tile
+    monkeypatch.setenv("H2O_ATTN_MODE", "fused")
     monkeypatch.setenv("H2O_ATTN_SPLIT", "4")
     cfg = _cfg(0, name="split-odd", B=1, Hq=6, Hkv=2, d=128, M=1000, R=90, T=1000 + 4 * 200 + 77,
                P=1000, S=200, dtype=torch.bfloat16, planted=0.02)
     run_stream(h2o, cfg)
+
+
+@pytest.mark.parametrize("case", ["ragged", "gqa8", "odd-tiles", "decode", "m2k-fused"])
+def test_stream_and_fused_paths(h2o, monkeypatch, case):
+    # the two tensor-core paths on shapes that stress the stream partition: ragged
+    # prefill and chunks, B > 1, an odd number of query heads per KV head (no head B
+    # in the last pair), units whose last pair has one tile, single-token steps; and
+    # the one-kernel path at the size where the stream path is the default
+    mode = "fused" if case == "m2k-fused" else "stream"
+    monkeypatch.setenv("H2O_ATTN_MODE", mode)
+    bf = dict(dtype=torch.bfloat16, d=128)
+    cfgs = {
+        "ragged": _cfg(0, name="stream-ragged", B=2, Hq=6, Hkv=2, M=300, R=17, T=100 + 37 * 7 + 11,
+                       P=100, S=37, planted=0.02, **bf),
+        "gqa8": _cfg(0, name="stream-gqa8", B=1, Hq=8, Hkv=1, M=520, R=40, T=520 + 3 * 260, P=520,
+                     S=260, planted=0.01, **bf),
+        "odd-tiles": _cfg(0, name="stream-odd", B=1, Hq=6, Hkv=2, M=1000, R=90, T=1000 + 4 * 200 + 77,
+                          P=1000, S=200, planted=0.02, **bf),
+        "decode": _cfg(0, name="stream-decode", M=72, R=5, T=72 + 30, P=72, S=1, **bf),
+        "m2k-fused": _cfg(1),
+    }
+    cfg = cfgs[case]
+    T = cfg.P + 3 * cfg.S if case == "m2k-fused" else None
+    s = run_stream(h2o, cfg, T=T, heads=[(0, 1), (0, 6)] if case == "m2k-fused" else None)
+    assert s["chunks"] >= 2
 
 
 def test_small_chunks_s128(h2o):
@@ -309,8 +336,7 @@ def test_fused_tail_matches_split_kernels(h2o, monkeypatch, base, kw, T):
             of = fused.step(q, k, v)
             monkeypatch.setenv("H2O_SPLIT_TAIL", "1")
             os_ = split.step(q, k, v)
-        assert fused.info()["launches"] == 2
-        assert split.info()["launches"] == 4
+        assert split.info()["launches"] - fused.info()["launches"] == 2
         assert torch.equal(of, os_), f"chunk {ci}: outputs differ"
         for x, y in zip(fused.read_state() + fused.read_delta(), split.read_state() + split.read_delta()):
             assert torch.equal(x, y), f"chunk {ci}: state differs"
