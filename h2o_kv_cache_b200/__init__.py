@@ -138,8 +138,10 @@ class H2OCache:
         self._chk(lib.h2o_info(self._h, arr))
         return {"B": arr[0], "t0": arr[1], "n_valid": arr[2], "last_S": arr[3], "launches": arr[4]}
 
-    def set_profiling(self, on: bool):
-        self._chk(lib.h2o_set_profiling(self._h, 1 if on else 0))
+    def set_profiling(self, on: bool, restart: bool = True):
+        """Per-kernel CUDA events on (restarting or continuing the count of
+        profiled steps) or off."""
+        self._chk(lib.h2o_set_profiling(self._h, (1 if restart else 2) if on else 0))
 
     def last_timings(self, age: int = 0):
         """ms of [attention, tail (score accumulate + select + scatter)] of the

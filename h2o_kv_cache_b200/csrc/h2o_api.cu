@@ -520,8 +520,9 @@ int h2o_info(h2o_t h, int64_t out[5]) {
 int h2o_set_profiling(h2o_t h, int on) {
   if (!h) return fail(nullptr, H2O_EINVAL, "h2o_set_profiling: NULL handle");
   if (on && !h->prefilled) return fail(h, H2O_ESTATE, "h2o_set_profiling: prefill first");
+  if (on < 0 || on > 2) return fail(h, H2O_EINVAL, "h2o_set_profiling: on must be 0, 1 or 2");
   h->prof = on != 0;
-  h->prof_steps = 0;
+  if (on == 1) h->prof_steps = 0;
   return H2O_OK;
 }
 

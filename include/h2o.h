@@ -129,11 +129,15 @@ int h2o_read_kv(h2o_t h, void* k_cache, void* v_cache, void* stream);
  * device kernels launched by the last step (or prefill).                      */
 int h2o_info(h2o_t h, int64_t out[5]);
 
-/* Per-kernel timing.  When on (default off; turning it on restarts the count),
- * each step records CUDA events around its kernels on the caller's stream,
- * into a ring that holds the last 64 steps, so steps can be enqueued back to
- * back and read afterwards.  h2o_step_timings() waits for the events of the
- * step `age` steps before the last (age 0 = the last step) and writes up to n
+/* Per-kernel timing.  on = 1 turns it on and restarts the count of profiled
+ * steps, on = 2 turns it on and keeps the count, on = 0 turns it off (the
+ * default).  While on, each step records CUDA events around its kernels on the
+ * caller's stream, into a ring that holds the last 64 profiled steps, so steps
+ * can be enqueued back to back and read afterwards.  The events sit between
+ * the step's kernels and so keep the next kernel from starting while the
+ * previous one drains (programmatic dependent launch).  h2o_step_timings()
+ * waits for the events of the profiled step `age` profiled steps before the
+ * last (age 0 = the last) and writes up to n
  * durations in milliseconds:
  *   ms[0] attention + summed weights, ms[1] the tail: score accumulate,
  *   select and scatter (one fused launch, or three kernels when the fused one
