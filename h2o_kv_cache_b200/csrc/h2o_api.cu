@@ -241,10 +241,15 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
     dout = h->st_out.p;
   }
 
+  // chunks of a few tokens (G * S <= 16 rows per KV head) take the decode
+  // kernel, which writes one partial row per KV head; forcing a tensor-core
+  // path (H2O_ATTN_MODE) bypasses it
+  const bool decode = h2o::decode_supported(h->G, S) && attn_mode() == 0;
   // scratch sized for this chunk
-  const int n_rt = (int)((S + h->row_tile - 1) / h->row_tile);
+  const int row_tile = decode ? (int)S : h->row_tile;
+  const int n_rt = decode ? 1 : (int)((S + h->row_tile - 1) / h->row_tile);
   const int64_t stride = h2o::partial_stride(h->M, S);
-  const int n_grp = h2o::partial_groups(h->G, h->use_umma);
+  const int n_grp = decode ? 1 : h2o::partial_groups(h->G, h->use_umma);
   const size_t part_bytes = (size_t)BH * n_grp * n_rt * stride * sizeof(float);
   H2O_CUDA(h, ensure(h->partials, part_bytes), "scratch alloc");
   H2O_CUDA(h, ensure(h->freed, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
@@ -276,7 +281,28 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   if (fault_injected("launch")) return fail(h, H2O_ECUDA, "injected launch failure");
   cudaError_t e = cudaSuccess;
   int launches = 1;
-  if (h->use_umma) {
+  if (decode) {
+    h2o::DecodeArgs da;
+    da.q = dq;
+    da.k = dk;
+    da.v = dv;
+    da.out = dout;
+    da.kcache = h->kc;
+    da.vcache = h->vc;
+    da.partials = static_cast<float*>(h->partials.p);
+    da.err = h->err;
+    da.B = h->B;
+    da.Hq = h->Hq;
+    da.Hkv = h->Hkv;
+    da.G = h->G;
+    da.d = h->d;
+    da.S = S;
+    da.M = h->M;
+    da.n_valid = h->n_valid;
+    da.stride = stride;
+    da.scale_log2 = a.scale * 1.4426950408889634f;
+    e = h2o::launch_decode(da, h->dtype, BH, true, st);
+  } else if (h->use_umma) {
     if (h->n_sm == 0) H2O_CUDA(h, cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device),
                                "device attribute");
     const int mode = attn_mode();
@@ -328,7 +354,7 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
     t.stride = stride;
     t.n_grp = n_grp;
     t.n_rt = n_rt;
-    t.row_tile = h->row_tile;
+    t.row_tile = row_tile;
     t.row_vecs = (int)(h->d * es / 16);
     e = h2o::launch_tail(t, BH, h->tail_cs, true, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "tail launch");
@@ -337,7 +363,7 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
     H2O_CUDA(h, ensure(h->newscore, (size_t)BH * S * sizeof(float)), "scratch alloc");
     e = h2o::launch_score_reduce(static_cast<float*>(h->partials.p), h->scores,
                                  static_cast<float*>(h->newscore.p), BH, n_grp, S, h->M,
-                                 h->n_valid, h->row_tile, stride, st);
+                                 h->n_valid, row_tile, stride, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "score reduce launch");
     e = h2o::launch_select(h->scores, h->pos, BH, h->M, h->t0, h->R, need, h->n_valid, S,
                            static_cast<int32_t*>(h->freed.p), S, h->err, st);

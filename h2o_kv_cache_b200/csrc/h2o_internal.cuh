@@ -119,6 +119,27 @@ struct TailArgs {
 int tail_cluster_size(int64_t M, int64_t S, int BH);
 cudaError_t launch_tail(const TailArgs& a, int BH, int cs, bool pdl, cudaStream_t st);
 
+// Chunks of a few tokens (G * S <= 16 query rows per KV head): attention with
+// summed weights by FMA dot products over a key split (decode.cu).  Column
+// sums go to ONE partial row per (b, KV head): partials [BH][stride].
+struct DecodeArgs {
+  const void* q;        // [B, Hq, S, d]
+  const void* k;        // [B, Hkv, S, d]
+  const void* v;        // [B, Hkv, S, d]
+  void* out;            // [B, Hq, S, d] or nullptr
+  const void* kcache;   // [B, Hkv, M, d]
+  const void* vcache;   // [B, Hkv, M, d]
+  float* partials;      // [B * Hkv, stride]
+  int* err;
+  int B, Hq, Hkv, G, d;
+  int64_t S, M, n_valid, stride;
+  float scale_log2;     // log2(e) / sqrt(d)
+  int kc = 1;           // CTAs per cluster (set by launch_decode)
+  int64_t per = 0;      // keys per CTA (set by launch_decode)
+};
+bool decode_supported(int G, int64_t S);
+cudaError_t launch_decode(DecodeArgs a, int dtype, int BH, bool pdl, cudaStream_t st);
+
 // Records msg as this thread's last error (h2o_last_error(NULL)); returns code.
 int set_thread_error(int code, const char* msg);
 

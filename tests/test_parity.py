@@ -203,6 +203,26 @@ def test_stream_and_fused_paths(h2o, monkeypatch, case):
     assert s["chunks"] >= 2
 
 
+@pytest.mark.parametrize("S,dtype,d", [(1, torch.bfloat16, 128), (2, torch.bfloat16, 128),
+                                       (4, torch.bfloat16, 64), (1, torch.float32, 64),
+                                       (3, torch.float32, 128)])
+def test_decode_kernel_small_chunks(h2o, S, dtype, d):
+    # G * S <= 16 rows per KV head: the key-split FMA kernel (G = 4 here), a ragged
+    # cache that fills and then evicts every step
+    cfg = _cfg(0, name=f"decode-{S}-{d}", B=2, Hq=8, Hkv=2, d=d, M=150, R=9, P=100, S=S,
+               T=100 + 60 * S + (S > 1), dtype=dtype, planted=0.02)
+    s = run_stream(h2o, cfg)
+    assert s["chunks"] >= 60
+
+
+def test_decode_kernel_m2k_and_m32k(h2o):
+    # decode steps on the benchmark caches: every key split over a cluster
+    cfg = _cfg(1, name="m2k-decode", S=1)
+    run_stream(h2o, cfg, heads=[(0, 0), (0, 7)], T=cfg.P + 40)
+    cfg = _cfg(3, name="m32k-decode", S=1)
+    run_stream(h2o, cfg, heads=[(0, 3)], T=cfg.P + 6, kv_check=False)
+
+
 def test_small_chunks_s128(h2o):
     # S = 128: 16 units for 148 SMs, so the kernel splits each unit's keys
     cfg = _cfg(1, name="m2k-s128", S=128)
