@@ -3,6 +3,7 @@
 // The operation each call performs is documented in include/h2o.h.
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -202,6 +203,11 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
 
   int rc = check_device_error(h, sync_check_enabled());
   if (rc != H2O_OK) return rc;
+
+  // token positions are stored as int32
+  if (h->t0 + S > (int64_t)INT32_MAX)
+    return fail(h, H2O_ESHAPE, "the stream would pass 2^31 - 1 tokens (t0=%lld, S=%lld)",
+                (long long)h->t0, (long long)S);
 
   // need and eligibility are fixed by the bookkeeping: the min(R, t0) most
   // recent tokens are always cached and protected, the rest of the valid slots

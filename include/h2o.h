@@ -60,7 +60,8 @@ typedef struct h2o_ctx* h2o_t;
 typedef enum {
   H2O_OK = 0,
   H2O_EINVAL = -1,   /* bad argument (null pointer, dtype, d, Hq % Hkv, R >= M) */
-  H2O_ESHAPE = -2,   /* shape cannot be served: P > M, S > M, or fewer evictable slots than needed */
+  H2O_ESHAPE = -2,   /* shape cannot be served: P > M, S > M, fewer evictable slots than needed,
+                        or a stream past 2^31 - 1 tokens (positions are int32) */
   H2O_ESTATE = -3,   /* step before prefill, prefill twice */
   H2O_ENOMEM = -4,   /* a device or pinned allocation failed */
   H2O_ECUDA = -5,    /* a CUDA runtime call or kernel launch failed */
