@@ -29,7 +29,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "H2O chunk-step query-tokens/s"
-PROF_EVERY = 4     # timed steps per step with per-kernel events
+PROF_EVERY = 8     # timed steps per step with per-kernel events
 UNIT = "query-tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -395,7 +395,7 @@ def sources_sha(names):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=24)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
