@@ -187,7 +187,47 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
   const int64_t s_end = hi < nv ? hi : nv;      // slots with partial columns
   const int64_t n_sr = (nloc + 4 * kLanes - 1) / (4 * kLanes);
   const int64_t n_cr = hi_s > lo_s ? (hi_s - lo_s + kLanes - 1) / kLanes : 0;
-  const int64_t rounds = n_sr > n_cr ? n_sr : n_cr;
+  // With at most kQuarters rows every run of a column's row list holds at most
+  // one row, and the run order is the plain sequential sum: a thread then takes
+  // whole columns (4 slots at a time), with no combine through shared memory.
+  const bool narrow = n_rows <= kQuarters;
+  if (narrow) {
+    for (int64_t s0 = lo + 4 * (int64_t)tid; s0 < hi; s0 += 4 * (int64_t)nthr) {
+      float scv[4] = {0.f, 0.f, 0.f, 0.f};
+      int32_t psv[4] = {-1, -1, -1, -1};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (s0 + e < hi) {
+          scv[e] = sc[s0 + e];
+          psv[e] = ps[s0 + e];
+        }
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (s0 < s_end)
+        for (int r = 0; r < n_rows; ++r)
+          add4(acc, __ldg(reinterpret_cast<const float4*>(base + s0 + (int64_t)r * p.stride)));
+      const float add[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t s = s0 + e;
+        if (s >= hi) break;
+        float v = scv[e];
+        if (s < nv) {
+          v += add[e];
+          sc[s] = v;
+        }
+        const int32_t q = psv[e];
+        keys[s - lo] = (q >= 0 && q < lim) ? ((uint64_t)ordered_bits(v) << 32) | (uint32_t)q : kNoKey;
+      }
+    }
+    for (int64_t i = lo_s + tid; i < hi_s; i += nthr) {
+      const int rt0 = (int)(i / p.row_tile);      // chunk key i is seen by row tiles rt >= rt0
+      float acc = 0.f;
+      for (int g = 0; g < p.n_grp; ++g)
+        for (int rt = rt0; rt < p.n_rt; ++rt) acc += __ldg(base + (int64_t)(g * p.n_rt + rt) * p.stride + M + i);
+      ns[i - lo_s] = acc;
+    }
+  }
+  const int64_t rounds = narrow ? 0 : (n_sr > n_cr ? n_sr : n_cr);
   for (int64_t rd = 0; rd < rounds; ++rd) {
     const int64_t s0 = lo + rd * 4 * kLanes + 4 * ln;
     float scv[4] = {0.f, 0.f, 0.f, 0.f};
@@ -357,27 +397,31 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
   __syncthreads();
   const bool sel_ok = need == 0 || (state == 1 && (int64_t)sh_tot == need);
   int32_t* fr = p.freed + bh * S;
+  int32_t* ev = p.evicted + bh * S;   // the delta record: the position each filled slot held
   if (do_sel) {
     int64_t o = (int64_t)sh_off + my_off;
     for (int64_t j = j0; j < j1; ++j) {
       const uint64_t key = keys[j];
       if (key != kNoKey && (key & mask) <= prefix) {
-        if (o < need) fr[o] = (int32_t)(lo + j);
+        if (o < need) {
+          fr[o] = (int32_t)(lo + j);
+          ev[o] = (int32_t)(uint32_t)key;   // the key's low word is the slot's position
+        }
         ++o;
       }
     }
   }
   if (rank == 0 && tid == 0 && !sel_ok) atomicOr(p.err, kErrSelect);
-  for (int64_t e = (int64_t)rank * nthr + tid; e < S - need; e += (int64_t)cs * nthr)
+  for (int64_t e = (int64_t)rank * nthr + tid; e < S - need; e += (int64_t)cs * nthr) {
     fr[need + e] = (int32_t)(nv + e);
+    ev[need + e] = -1;
+  }
   cluster_sync();   // the freed list is complete; rank 0's shared memory is no longer read
 
   // ---- 4. chunk row i -> slot fr[i]: K and V rows, pos = t0 + i, initial score
   if (!sel_ok) return;
-  // old = the position the slot held: lane j read it with the slot of row j
-  auto finish_row = [&](int64_t i, int32_t slot, int32_t old) {
+  auto finish_row = [&](int64_t i, int32_t slot) {
     if (lane == 0) {
-      p.evicted[bh * S + i] = old;                      // the delta record of this chunk row
       p.pos[bh * M + slot] = (int32_t)(p.t0 + i);
       p.scores[bh * M + slot] = ns[i - lo_s];
     }
@@ -386,43 +430,59 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
   if (pre_ok) {
     // lane k fetches the slot of the warp's k-th row
     const int32_t my_slot = lane < n_mine ? ld_relaxed(fr + lo_s + warp + (int64_t)lane * nwarps) : -1;
-    const int32_t my_old = (my_slot >= 0 && my_slot < M) ? p.pos[bh * M + my_slot] : -1;
 #pragma unroll
     for (int k = 0; k < kPre; ++k) {
       if (k < n_mine) {
         const int64_t i = lo_s + warp + (int64_t)k * nwarps;
         const int32_t slot = __shfl_sync(0xffffffffu, my_slot, k);
-        const int32_t old = __shfl_sync(0xffffffffu, my_old, k);
         if (slot < 0 || slot >= M) {
           if (lane == 0) atomicOr(p.err, kErrBounds);
         } else {
           const int64_t dst = (bh * M + slot) * rv;
           if (lane < rv) p.kc[dst + lane] = pre[k];
           else if (lane < vecs2) p.vc[dst + lane - rv] = pre[k];
-          finish_row(i, slot, old);
+          finish_row(i, slot);
         }
       }
     }
     k_from = kPre;
   }
+  // the rest of the warp's rows, eight at a time: their loads in flight together
   for (int64_t k0 = k_from; k0 < n_mine; k0 += 32) {
     const int32_t my_slot = k0 + lane < n_mine ? ld_relaxed(fr + lo_s + warp + (k0 + lane) * nwarps) : -1;
-    const int32_t my_old = (my_slot >= 0 && my_slot < M) ? p.pos[bh * M + my_slot] : -1;
     const int kn = n_mine - k0 < 32 ? (int)(n_mine - k0) : 32;
-    for (int jj = 0; jj < kn; ++jj) {
-      const int64_t i = lo_s + warp + (k0 + jj) * nwarps;
-      const int32_t slot = __shfl_sync(0xffffffffu, my_slot, jj);
-      const int32_t old = __shfl_sync(0xffffffffu, my_old, jj);
-      if (slot < 0 || slot >= M) {
-        if (lane == 0) atomicOr(p.err, kErrBounds);
-        continue;
+    for (int jb = 0; jb < kn; jb += 8) {
+      uint4 buf[8][2];                                   // a row is at most 64 vectors
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (jb + u < kn) {
+          const int64_t src = (bh * S + lo_s + warp + (k0 + jb + u) * nwarps) * rv;
+#pragma unroll
+          for (int hv = 0; hv < 2; ++hv) {
+            const int c = lane + 32 * hv;                // K row then V row
+            if (c < vecs2) buf[u][hv] = c < rv ? __ldg(p.k + src + c) : __ldg(p.v + src + c - rv);
+          }
+        }
       }
-      const int64_t src = (bh * S + i) * rv, dst = (bh * M + slot) * rv;
-      for (int c = lane; c < vecs2; c += 32) {   // K row then V row
-        if (c < rv) p.kc[dst + c] = __ldg(p.k + src + c);
-        else p.vc[dst + c - rv] = __ldg(p.v + src + c - rv);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (jb + u < kn) {
+          const int64_t i = lo_s + warp + (k0 + jb + u) * nwarps;
+          const int32_t slot = __shfl_sync(0xffffffffu, my_slot, jb + u);
+          if (slot < 0 || slot >= M) {
+            if (lane == 0) atomicOr(p.err, kErrBounds);
+          } else {
+            const int64_t dst = (bh * M + slot) * rv;
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {
+              const int c = lane + 32 * hv;
+              if (c < rv) p.kc[dst + c] = buf[u][hv];
+              else if (c < vecs2) p.vc[dst + c - rv] = buf[u][hv];
+            }
+            finish_row(i, slot);
+          }
+        }
       }
-      finish_row(i, slot, old);
     }
   }
 }
