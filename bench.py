@@ -62,15 +62,62 @@ def select_scatter_bytes(cfg, S):
     return state + rows
 
 
+CLOCK_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown"}   # NVML clock-event reason bits
+
+
+def clock_poller(index, period_s=0.0005):
+    """Child process of ClockSampler: polls NVML every period_s until its standard
+    input closes, then prints one JSON line of (SM MHz, reason bits) samples.  A
+    process of its own, so that the bench's Python thread never delays it."""
+    import threading
+    import pynvml as nv
+    nv.nvmlInit()
+    hdl = nv.nvmlDeviceGetHandleByIndex(index)
+    smax = nv.nvmlDeviceGetMaxClockInfo(hdl, nv.NVML_CLOCK_SM)
+    done = threading.Event()
+    threading.Thread(target=lambda: (sys.stdin.read(), done.set()), daemon=True).start()
+    print("ready", flush=True)
+    samples = []
+    while not done.is_set():
+        try:
+            samples.append((nv.nvmlDeviceGetClockInfo(hdl, nv.NVML_CLOCK_SM),
+                            int(nv.nvmlDeviceGetCurrentClocksThrottleReasons(hdl))))
+        except Exception:  # noqa: BLE001 - a failed sample is skipped
+            pass
+        time.sleep(period_s)
+    print(json.dumps({"max": smax, "samples": samples}), flush=True)
+
+
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    """SM clock and clock-event (throttle) reasons sampled during a region.
+
+    A child process polls NVML every 0.5 ms from __enter__ to __exit__ (the timed
+    steps run for tens of milliseconds, far shorter than nvidia-smi's sampling
+    period); without NVML, nvidia-smi samples every 100 ms instead."""
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.nvml = None
+        self.result = None
+        self.source = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
 
     def __enter__(self):
+        try:
+            import pynvml  # noqa: F401 - only probes that NVML is importable
+            self.nvml = subprocess.Popen(
+                [sys.executable, os.path.abspath(__file__), "--clock-poller", str(self.index)],
+                stdin=subprocess.PIPE, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            if self.nvml.stdout.readline().strip() == "ready":
+                self.source = "nvml, 0.5 ms"
+                return self
+            self.nvml.kill()
+            self.nvml.wait()
+        except (ImportError, OSError):
+            pass
+        self.nvml = None
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
@@ -82,11 +129,19 @@ class ClockSampler:
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
+            self.source = "nvidia-smi, 100 ms"
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
 
     def __exit__(self, *exc):
+        if self.nvml is not None:
+            try:
+                out, _ = self.nvml.communicate(timeout=10)
+                self.result = json.loads(out.strip().splitlines()[-1])
+            except (subprocess.TimeoutExpired, ValueError, IndexError):
+                self.nvml.kill()
+                self.nvml.wait()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -96,8 +151,17 @@ class ClockSampler:
             self.f.close()
 
     def summary(self):
+        if self.nvml is not None:
+            if self.result is None:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock poller failed"]}
+            smp = self.result["samples"]
+            sm = [float(m) for m, _ in smp]
+            reasons = sorted({n for _, b in smp for bit, n in CLOCK_REASONS.items() if b & bit})
+            return {"sm_mhz": statistics.median(sm) if sm else None,
+                    "sm_max_mhz": float(self.result["max"]), "reasons": reasons,
+                    "samples": len(sm), "source": self.source}
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
@@ -114,7 +178,7 @@ class ClockSampler:
                     if v.lower() == "active":
                         reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 def dist_setup(n_gpus):
@@ -301,13 +365,13 @@ def run_ours(args, cfg):
     h2d = d2h = 0
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+    pinned = {}                                    # one pinned host copy per distinct chunk
     host_steps = []
     for i in range(args.steps):
-        hs = []
-        for cache, chunks in layers:
-            q, k, v = chunks[1 + (ci + i) % n_avail]
-            hs.append(tuple(x.cpu().pin_memory() for x in (q, k, v)))
-        host_steps.append(hs)
+        j = 1 + (ci + i) % n_avail
+        if j not in pinned:
+            pinned[j] = [tuple(x.cpu().pin_memory() for x in chunks[j]) for _, chunks in layers]
+        host_steps.append(pinned[j])
     h2d = sum(x.numel() * x.element_size() for hs in host_steps[0] for x in hs)
     d2h = hout.numel() * hout.element_size() * len(layers)
     barrier(world)
@@ -395,13 +459,17 @@ def sources_sha(names):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=24)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--clock-poller", type=int, default=None, help=argparse.SUPPRESS)
     args = ap.parse_args()
+    if args.clock_poller is not None:
+        clock_poller(args.clock_poller)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from h2o_kv_cache_b200.workload import CONFIGS
