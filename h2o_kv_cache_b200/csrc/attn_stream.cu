@@ -42,7 +42,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kA_OffQ = 0;
 constexpr uint32_t kA_OffK = 2 * kTile;
 constexpr uint32_t kA_Slot = 2 * kTile;
-constexpr uint32_t kA_OffBar = kA_OffK + 2 * kA_Slot;
+// the two softmax warpgroups' (max, sum) halves of a piece's rows, [2][128] float2
+constexpr uint32_t kA_OffMrg = kA_OffK + 2 * kA_Slot;
+constexpr uint32_t kA_OffBar = kA_OffMrg + 2 * BM * 8;
 enum { A_Q = 0, A_Q_EMPTY, A_K_FULL, A_K_EMPTY = A_K_FULL + 2, A_S_FULL = A_K_EMPTY + 2,
        A_S_EMPTY = A_S_FULL + 2, A_DRAIN = A_S_EMPTY + 2, A_NUM = A_DRAIN + 1 };
 
@@ -159,7 +161,7 @@ lse_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < A_NUM; ++i)
-      mbar_init(bar(i), (i == A_S_EMPTY || i == A_S_EMPTY + 1) ? 128u : 1u);
+      mbar_init(bar(i), (i == A_S_EMPTY || i == A_S_EMPTY + 1) ? 256u : 1u);   // both warpgroups
     *abort_flag = 0;
     *n_pieces = build_pieces(p, pcs);
     fence_mbar_init();
@@ -266,15 +268,21 @@ lse_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else {
     // =========================================================== softmax: row (max, sum)
-    const int w = (warp - 2) >> 2;                    // 0: head A, 1: head B
+    // Both warpgroups read each head's S tile, warpgroup w taking keys
+    // [128 w, 128 w + 128) of every 256-key tile (a tile is released after a
+    // quarter of the work, so the next tile's MMA overlaps the other head's
+    // tile); thread = query row r of both heads.  At the end of a piece
+    // warpgroup w merges the two halves of head w's rows and writes them.
+    const int w = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                 // TMEM lane = query row
-    const uint32_t s_tmem = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)w * 256u;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)w * 128u;
     const float c = p.scale_log2;
     const int64_t S = p.S, nv = p.n_valid;
+    float2* mrg = reinterpret_cast<float2*>(sbase + kA_OffMrg);
     bool ok = true;
     int tc = 0;
-    for (int pi = 0; ok && pi < npc; ++pi) {
+    for (int pi = 0; pi < npc; ++pi) {
       const Piece x = pcs[pi];
       const UnitGeo g = unit_geo(p, x.u);
       const int64_t row_i = g.i0 + r;
@@ -286,28 +294,43 @@ lse_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int64_t lim = cache ? nv : row_lim;
         return (int)(lim - key0 > 64 ? 64 : (lim - key0 < 0 ? 0 : lim - key0));
       };
-      float m = -INFINITY, l = 0.f;
+      float mh[2] = {-INFINITY, -INFINITY}, lh[2] = {0.f, 0.f};
       for (int pr = x.a; ok && pr < x.c; ++pr) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(A_S_FULL + w), (uint32_t)tc & 1u, abort_flag, p.err,
-                                               kWaitLimitNs, kErrTimeout));
-        if (!ok) break;
-        tc_fence_after();
+#pragma unroll
+        for (int hw = 0; hw < 2; ++hw) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(A_S_FULL + hw), (uint32_t)tc & 1u, abort_flag, p.err,
+                                                 kWaitLimitNs, kErrTimeout));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t s_tmem = lane_base + (uint32_t)hw * 256u;
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t v[2][32];
-          tmem_ld32(s_tmem + ch * 64, v[0]);
-          tmem_ld32(s_tmem + ch * 64 + 32, v[1]);
-          tmem_wait_ld();
-          if (ch == 3) {
-            tc_fence_before();
-            mbar_arrive(bar(A_S_EMPTY + w));
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t v[2][32];
+            tmem_ld32(s_tmem + ch * 64, v[0]);
+            tmem_ld32(s_tmem + ch * 64 + 32, v[1]);
+            tmem_wait_ld();
+            if (ch == 1) {
+              tc_fence_before();
+              mbar_arrive(bar(A_S_EMPTY + hw));
+            }
+            row_chunk(v, nvis_of(2 * pr + w, ch), c, mh[hw], lh[hw]);
           }
-          row_chunk(v, nvis_of(2 * pr + (ch >> 1), ch & 1), c, m, l);
         }
         __syncwarp();
         ++tc;
       }
+      // warpgroup w takes the other warpgroup's half of head w's rows.  Every
+      // warp passes both barriers whatever its `ok`, and the second one makes
+      // the decision to stop the same for all of them.
+      mrg[(1 - w) * BM + r] = w ? make_float2(mh[0], lh[0]) : make_float2(mh[1], lh[1]);
+      named_bar_sync(1, 256);
+      const float2 o = mrg[w * BM + r];
+      ok = named_bar_and(1, 256, ok);   // both read: the next piece may overwrite the area
       if (!ok) break;
+      const float m_own = w ? mh[1] : mh[0], l_own = w ? lh[1] : lh[0];
+      const float m = fmaxf(m_own, o.x);
+      // an empty half has sum 0 (or NaN when its keys were all masked)
+      const float l = (l_own > 0.f ? l_own * ex2(m_own - m) : 0.f) + (o.y > 0.f ? o.y * ex2(o.x - m) : 0.f);
       p.ws_ml[((int64_t)x.u * p.maxp + x.k) * (2 * BM) + w * BM + r] = make_float2(m, l);
     }
   }
@@ -567,34 +590,40 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // chunk key `key` is seen by query columns q with i0 + q >= key
         const int qmin = cache ? 0 : (int)(key - g.i0 > 0 ? key - g.i0 : 0);
         const bool full = __all_sync(0xffffffffu, key_ok && qmin == 0);
-        float cs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[32];
+        uint64_t cs4[4] = {0ull, 0ull, 0ull, 0ull};
+        // both halves of the key's P^T row in registers before waiting for the
+        // buffer, so the previous tile's O^T MMA overlaps all the exponentials
+        uint32_t pk[32], pk2[32];
         {
           uint32_t v[2][32];
           tmem_ld32(st_tmem, v[0]);
           tmem_ld32(st_tmem + 32, v[1]);
           tmem_wait_ld();
-          if (full) key_half<true>(v, nl_w, c, key_ok, qmin, cs8, pk);
-          else key_half<false>(v, nl_w, c, key_ok, qmin, cs8, pk);
+          if (full) key_half<true>(v, nl_w, c, key_ok, qmin, cs4, pk);
+          else key_half<false>(v, nl_w, c, key_ok, qmin, cs4, pk);
         }
-        {
-          uint32_t v[2][32];
-          tmem_ld32(st_tmem + 64, v[0]);
-          tmem_ld32(st_tmem + 96, v[1]);
+        // the second half in two 32-query pieces: fewer registers live beside
+        // the packed first half
+#pragma unroll
+        for (int qc = 0; qc < 2; ++qc) {
+          uint32_t v[32];
+          tmem_ld32(st_tmem + 64 + qc * 32, v);
           tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(bar(B_ST_EMPTY));
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)st & 1u) ^ 1u, abort_flag,
-                                                 p.err, kWaitLimitNs, kErrTimeout));
-          if (!ok) break;
-          store_p_half(p_row, r, pk);
-          if (full) key_half<true>(v, nl_w + 64, c, key_ok, qmin - 64, cs8, pk);
-          else key_half<false>(v, nl_w + 64, c, key_ok, qmin - 64, cs8, pk);
-          store_p_half(p_row + kAtom, r, pk);
+          if (qc == 1) {
+            tc_fence_before();
+            mbar_arrive(bar(B_ST_EMPTY));
+          }
+          if (full) key_part<true, 32>(v, nl_w + 64 + qc * 32, c, key_ok, qmin - 64 - qc * 32, cs4, pk2 + qc * 16);
+          else key_part<false, 32>(v, nl_w + 64 + qc * 32, c, key_ok, qmin - 64 - qc * 32, cs4, pk2 + qc * 16);
         }
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)st & 1u) ^ 1u, abort_flag,
+                                               p.err, kWaitLimitNs, kErrTimeout));
+        if (!ok) break;
+        store_p_half(p_row, r, pk);
+        store_p_half(p_row + kAtom, r, pk2);
         fence_async_smem();
         mbar_arrive(bar(B_P_FULL));
-        const float cs = ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
+        const float cs = cs_total(cs4);
         if (w == 0) {
           prev_cs = cs;
           prev_part = part;

@@ -72,6 +72,10 @@ constexpr uint32_t kSmemUsed = kOffCs + BN * 4;
 // first overwrites only after every CTA of the cluster has read it
 constexpr uint32_t kOffX = kOffR + 2 * kSlot1;
 static_assert(kOffX >= kOffP && kOffX + 2 * BM * 8 <= kOffR + kRBytes, "exchange inside P^T's tail");
+// the two warpgroups' sweep-1 (max, sum) halves, [2][128] float2: right after
+// the exchange area, read before any P^T store (a barrier of both warpgroups)
+constexpr uint32_t kOffMrg = kOffX + 2 * BM * 8;
+static_assert(kOffMrg + 2 * BM * 8 <= kOffR + kRBytes, "merge area inside P^T's tail");
 constexpr int kMaxSplit = 8;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // slack for 1024-byte alignment
 static_assert(2 * kSlot1 <= kRBytes, "sweep-1 slots fit in R");
@@ -142,7 +146,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t cnt = 1;
-      if (i == B_S_EMPTY || i == B_S_EMPTY + 1) cnt = 128;   // one warpgroup
+      if (i == B_S_EMPTY || i == B_S_EMPTY + 1) cnt = 256;   // both warpgroups
       if (i == B_ST_EMPTY || i == B_P_FULL) cnt = 256;        // both warpgroups
       if (i == B_CS_FULL || i == B_CS_EMPTY) cnt = 128;       // one warpgroup
       if (i == B_X_READY || i == B_X_READ) cnt = (uint32_t)kc;  // one arrival per CTA
@@ -349,14 +353,17 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_NEVER), 0, abort_flag, p.err, 1000000ull, kErrTimeout));
     }
 
-    // ----- sweep 1: thread = query row i0 + r of head w; running (max, sum).
-    // The sum is kept against a reference max that is only raised when a
-    // 64-key chunk's max exceeds it by more than 8 (log2 units), so the
-    // exponentials of a chunk never wait for that chunk's max.
+    // ----- sweep 1: both warpgroups read each head's S tile, warpgroup w
+    // taking keys [128 w, 128 w + 128) of every 256-key tile, so a tile is
+    // released after a quarter of the work and the next tile's MMA overlaps
+    // the other head's tile.  Thread = query row i0 + r of both heads, with a
+    // running (max, sum) of each over its keys; the sum is kept against a
+    // reference max that is only raised when a 64-key chunk's max exceeds it
+    // by more than 8 (log2 units), so the exponentials of a chunk never wait
+    // for that chunk's max.
     const int64_t row_i = i0 + r;
     const int64_t row_lim = (row_i + 1 < S) ? row_i + 1 : S;   // chunk keys < row_lim are seen
-    float m = -INFINITY, l = 0.f;
-    const uint32_t s_tmem = lane_base + (uint32_t)w * 256u;
+    float mh[2] = {-INFINITY, -INFINITY}, lh[2] = {0.f, 0.f};
     auto nvis_of = [&](int t, int half64) -> int {
       const int tg = t_lo + t;
       if (tg >= t_hi) return 0;
@@ -366,31 +373,42 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       return (int)(lim - key0 > 64 ? 64 : (lim - key0 < 0 ? 0 : lim - key0));
     };
     for (int u = 0; ok && u < n1; ++u) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + w), (uint32_t)u & 1u, abort_flag, p.err,
-                                             kWaitLimitNs, kErrTimeout));
-      if (!ok) break;
-      tc_fence_after();
+#pragma unroll
+      for (int hw = 0; hw < 2; ++hw) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + hw), (uint32_t)u & 1u, abort_flag, p.err,
+                                               kWaitLimitNs, kErrTimeout));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t s_tmem = lane_base + (uint32_t)hw * 256u + (uint32_t)w * 128u;
 #pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {                 // keys 0-127 of the tile, 64 at a time
-        uint32_t v[2][32];
-        tmem_ld32(s_tmem + ch * 64, v[0]);
-        tmem_ld32(s_tmem + ch * 64 + 32, v[1]);
-        tmem_wait_ld();
-        row_chunk(v, nvis_of(2 * u, ch), c, m, l);
-      }
-#pragma unroll 1
-      for (int ch = 2; ch < 4; ++ch) {
-        uint32_t v[2][32];
-        tmem_ld32(s_tmem + ch * 64, v[0]);
-        tmem_ld32(s_tmem + ch * 64 + 32, v[1]);
-        tmem_wait_ld();
-        if (ch == 3) {
-          tc_fence_before();
-          mbar_arrive(bar(B_S_EMPTY + w));
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t v[2][32];
+          tmem_ld32(s_tmem + ch * 64, v[0]);
+          tmem_ld32(s_tmem + ch * 64 + 32, v[1]);
+          tmem_wait_ld();
+          if (ch == 1) {
+            tc_fence_before();
+            mbar_arrive(bar(B_S_EMPTY + hw));
+          }
+          row_chunk(v, nvis_of(2 * u + w, ch), c, mh[hw], lh[hw]);
         }
-        row_chunk(v, nvis_of(2 * u + 1, ch - 2), c, m, l);
       }
       __syncwarp();
+    }
+    // warpgroup w finishes head w's rows: it takes the other warpgroup's
+    // (max, sum) of them from shared memory.  Every warp passes both barriers
+    // whatever its `ok`, so a warp that aborted cannot leave the others waiting.
+    float m, l;
+    {
+      float2* mrg = reinterpret_cast<float2*>(sbase + kOffMrg);
+      mrg[(1 - w) * BM + r] = w ? make_float2(mh[0], lh[0]) : make_float2(mh[1], lh[1]);
+      named_bar_sync(4, 256);
+      const float2 o = mrg[w * BM + r];
+      const float m_own = w ? mh[1] : mh[0], l_own = w ? lh[1] : lh[0];
+      m = fmaxf(m_own, o.x);
+      // an empty half has sum 0 (or NaN when its keys were all masked)
+      l = (l_own > 0.f ? l_own * ex2(m_own - m) : 0.f) + (o.y > 0.f ? o.y * ex2(o.x - m) : 0.f);
+      named_bar_sync(4, 256);   // both read: P^T may overwrite the area
     }
     // negated base-2 log-sum-exp of each row; -inf zeroes rows past S and a missing head B
     if (kc == 1) {
@@ -463,15 +481,18 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // chunk key `key` is seen by query columns q with i0 + q >= key
       const int qmin = cache ? 0 : (int)(key - i0 > 0 ? key - i0 : 0);
       const bool full = __all_sync(0xffffffffu, key_ok && qmin == 0);
-      float cs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
+      uint64_t cs4[4] = {0ull, 0ull, 0ull, 0ull};
+      // both 64-query halves of this key's P^T row are formed in registers
+      // before waiting for the previous tile's O^T MMA to release the buffer,
+      // so that MMA overlaps all of this tile's exponentials
+      uint32_t pk[32], pk2[32];
       {
         uint32_t v[2][32];
         tmem_ld32(st_tmem, v[0]);
         tmem_ld32(st_tmem + 32, v[1]);
         tmem_wait_ld();
-        if (full) key_half<true>(v, nl_w, c, key_ok, qmin, cs8, pk);
-        else key_half<false>(v, nl_w, c, key_ok, qmin, cs8, pk);
+        if (full) key_half<true>(v, nl_w, c, key_ok, qmin, cs4, pk);
+        else key_half<false>(v, nl_w, c, key_ok, qmin, cs4, pk);
       }
       {
         uint32_t v[2][32];
@@ -480,24 +501,23 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(B_ST_EMPTY));
-        if (kc > 1 && j == 0) {   // the cluster is done with the exchange area
-          ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_X_READ), 0, abort_flag, p.err,
-                                                       kWaitLimitNs, kErrTimeout));
-          if (!ok) break;
-        }
-        // this warpgroup's P^T half of the previous tile has been read by its O^T MMA:
-        // store the first 64 queries now, the second half's exponentials overlap it
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
-                                               p.err, kWaitLimitNs, kErrTimeout));
-        if (!ok) break;
-        store_p_half(p_row, r, pk);
-        if (full) key_half<true>(v, nl_w + 64, c, key_ok, qmin - 64, cs8, pk);
-        else key_half<false>(v, nl_w + 64, c, key_ok, qmin - 64, cs8, pk);
-        store_p_half(p_row + kAtom, r, pk);
+        if (full) key_half<true>(v, nl_w + 64, c, key_ok, qmin - 64, cs4, pk2);
+        else key_half<false>(v, nl_w + 64, c, key_ok, qmin - 64, cs4, pk2);
       }
+      if (kc > 1 && j == 0) {   // the cluster is done with the exchange area
+        ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_X_READ), 0, abort_flag, p.err,
+                                                     kWaitLimitNs, kErrTimeout));
+        if (!ok) break;
+      }
+      // this warpgroup's P^T half of the previous tile has been read by its O^T MMA
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
+                                             p.err, kWaitLimitNs, kErrTimeout));
+      if (!ok) break;
+      store_p_half(p_row, r, pk);
+      store_p_half(p_row + kAtom, r, pk2);
       fence_async_smem();
       mbar_arrive(bar(B_P_FULL));
-      const float cs = ((cs8[0] + cs8[1]) + (cs8[2] + cs8[3])) + ((cs8[4] + cs8[5]) + (cs8[6] + cs8[7]));
+      const float cs = cs_total(cs4);
       if (w == 0) {
         prev_cs = cs;
         prev_col = key_ok ? (cache ? key : M + key) : -1;
