@@ -33,32 +33,39 @@ namespace {
 using namespace sm100;
 using namespace attn;
 
-constexpr int kThreads = 320;
+constexpr int kWg = 4;                           // softmax warpgroups (both kernels)
+constexpr int kSoft = 128 * kWg;                 // softmax threads
+constexpr int kThreads = 64 + kSoft;             // + TMA producer warp + MMA warp
+static_assert(kWg == kStreamRows, "one partial row per softmax warpgroup");
 constexpr int kMaxPieces = 8;                    // per CTA (the host checks)
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kDescHi = desc_hi_sw128(1024);   // 8 rows of 128 bytes between core-matrix groups
 
 // kernel A shared memory: Q, two 64 KB slots of 256 keys
 constexpr uint32_t kA_OffQ = 0;
 constexpr uint32_t kA_OffK = 2 * kTile;
 constexpr uint32_t kA_Slot = 2 * kTile;
-// the two softmax warpgroups' (max, sum) halves of a piece's rows, [2][128] float2
+// the softmax warpgroups' (max, sum) over their keys of a piece's rows,
+// [warpgroup][head][128] float2
 constexpr uint32_t kA_OffMrg = kA_OffK + 2 * kA_Slot;
-constexpr uint32_t kA_OffBar = kA_OffMrg + 2 * BM * 8;
+constexpr uint32_t kA_OffBar = kA_OffMrg + kWg * 2 * BM * 8;
 enum { A_Q = 0, A_Q_EMPTY, A_K_FULL, A_K_EMPTY = A_K_FULL + 2, A_S_FULL = A_K_EMPTY + 2,
        A_S_EMPTY = A_S_FULL + 2, A_DRAIN = A_S_EMPTY + 2, A_NUM = A_DRAIN + 1 };
 
 // kernel B shared memory: Q, a ring of three 32 KB K / V slots, P^T (64 KB),
-// the rows' negated log-sum-exp, head B's column sums of a tile
+// the rows' negated log-sum-exp
 constexpr int NS2 = 3;
 constexpr uint32_t kB_OffQ = 0;
 constexpr uint32_t kB_OffR = 2 * kTile;
 constexpr uint32_t kB_OffP = kB_OffR + NS2 * kTile;
 constexpr uint32_t kB_OffLse = kB_OffP + 2 * kTile;
-constexpr uint32_t kB_OffCs = kB_OffLse + 2 * BM * 4;
-constexpr uint32_t kB_OffBar = kB_OffCs + BN * 4;
+constexpr uint32_t kB_OffBar = kB_OffLse + 2 * BM * 4;
+// S^T is two buffers of 128 columns, one per head (TMEM columns 0-127: head
+// A's queries, 128-255: head B's), each with its own full / empty barriers,
+// so the softmax reads one head's tile while the other head's MMA runs
 enum { B_Q = 0, B_Q_EMPTY, B_R_FULL, B_R_EMPTY = B_R_FULL + NS2, B_ST_FULL = B_R_EMPTY + NS2,
-       B_ST_EMPTY, B_P_FULL, B_P_EMPTY, B_O_FULL, B_O_EMPTY, B_CS_FULL, B_CS_EMPTY, B_DRAIN,
+       B_ST_EMPTY = B_ST_FULL + 2, B_P_FULL = B_ST_EMPTY + 2, B_P_EMPTY, B_O_FULL, B_O_EMPTY, B_DRAIN,
        B_NUM };
 
 // after the barriers: TMEM address, abort flag, the CTA's pieces
@@ -80,6 +87,7 @@ struct SParams {
   float* ws_o;          // [units][maxp][2 * BM][D]: a piece's partial O (split units)
   int* count;           // [units]: pieces of the unit done with sweep 2
   int B, Hq, Hkv, G, n_pg, n_rt, maxp;
+  int n_grp;            // partial rows per (b, KV head, row tile): kStreamRows per head pair
   int64_t S, M, n_valid, stride;
   int64_t total_pairs;  // over all units
   float scale_log2;
@@ -161,7 +169,7 @@ lse_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < A_NUM; ++i)
-      mbar_init(bar(i), (i == A_S_EMPTY || i == A_S_EMPTY + 1) ? 256u : 1u);   // both warpgroups
+      mbar_init(bar(i), (i == A_S_EMPTY || i == A_S_EMPTY + 1) ? 128u * kWg : 1u);   // every softmax thread
     *abort_flag = 0;
     *n_pieces = build_pieces(p, pcs);
     fence_mbar_init();
@@ -249,12 +257,11 @@ lse_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                            kWaitLimitNs, kErrTimeout);
             if (!ok) break;
             tc_fence_after();
+            const uint32_t a0 = desc_lo(q_addr + (uint32_t)w * kAtom, 16), b0 = desc_lo(k_addr, 16);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t da = smem_desc_sw128(q_addr + (uint32_t)w * kAtom + kmajor_off(kk, 256), 16, 1024);
-              const uint64_t db = smem_desc_sw128(k_addr + kmajor_off(kk, 256), 16, 1024);
-              umma_bf16(tmem + (uint32_t)w * 256u, da, db, idesc, kk > 0 ? 1u : 0u);
-            }
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_bf16(tmem + (uint32_t)w * 256u, a0 + (kmajor_off(kk, 256) >> 4), kDescHi,
+                        b0 + (kmajor_off(kk, 256) >> 4), kDescHi, idesc, kk > 0 ? 1u : 0u);
             umma_commit(bar(A_S_FULL + w));
           }
           if (ok) umma_commit(bar(A_K_EMPTY + s));
@@ -268,15 +275,16 @@ lse_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else {
     // =========================================================== softmax: row (max, sum)
-    // Both warpgroups read each head's S tile, warpgroup w taking keys
-    // [128 w, 128 w + 128) of every 256-key tile (a tile is released after a
-    // quarter of the work, so the next tile's MMA overlaps the other head's
-    // tile); thread = query row r of both heads.  At the end of a piece
-    // warpgroup w merges the two halves of head w's rows and writes them.
-    const int w = (warp - 2) >> 2;
+    // Four warpgroups read each head's S tile, warpgroup g taking keys
+    // [64 g, 64 g + 64) of every 256-key tile (four warps per SM sub-partition
+    // hide each other's latencies; a tile is released as soon as it is loaded
+    // into registers); thread = query row r of both heads.  At the end of a
+    // piece warpgroup w < 2 merges the four (max, sum) of head w's rows, in
+    // warpgroup order, and writes them.
+    const int wg = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                 // TMEM lane = query row
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)w * 128u;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)wg * 64u;
     const float c = p.scale_log2;
     const int64_t S = p.S, nv = p.n_valid;
     float2* mrg = reinterpret_cast<float2*>(sbase + kA_OffMrg);
@@ -302,36 +310,38 @@ lse_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                                  kWaitLimitNs, kErrTimeout));
           if (!ok) break;
           tc_fence_after();
-          const uint32_t s_tmem = lane_base + (uint32_t)hw * 256u;
-#pragma unroll 1
-          for (int ch = 0; ch < 2; ++ch) {
-            uint32_t v[2][32];
-            tmem_ld32(s_tmem + ch * 64, v[0]);
-            tmem_ld32(s_tmem + ch * 64 + 32, v[1]);
-            tmem_wait_ld();
-            if (ch == 1) {
-              tc_fence_before();
-              mbar_arrive(bar(A_S_EMPTY + hw));
-            }
-            row_chunk(v, nvis_of(2 * pr + w, ch), c, mh[hw], lh[hw]);
-          }
+          uint32_t v[2][32];
+          tmem_ld32(lane_base + (uint32_t)hw * 256u, v[0]);
+          tmem_ld32(lane_base + (uint32_t)hw * 256u + 32u, v[1]);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(A_S_EMPTY + hw));
+          row_chunk(v, nvis_of(2 * pr + (wg >> 1), wg & 1), c, mh[hw], lh[hw]);
         }
         __syncwarp();
         ++tc;
       }
-      // warpgroup w takes the other warpgroup's half of head w's rows.  Every
-      // warp passes both barriers whatever its `ok`, and the second one makes
-      // the decision to stop the same for all of them.
-      mrg[(1 - w) * BM + r] = w ? make_float2(mh[0], lh[0]) : make_float2(mh[1], lh[1]);
-      named_bar_sync(1, 256);
-      const float2 o = mrg[w * BM + r];
-      ok = named_bar_and(1, 256, ok);   // both read: the next piece may overwrite the area
+      // Every warp passes both barriers whatever its `ok`, and the second one
+      // makes the decision to stop the same for all of them.
+      mrg[(wg * 2 + 0) * BM + r] = make_float2(mh[0], lh[0]);
+      mrg[(wg * 2 + 1) * BM + r] = make_float2(mh[1], lh[1]);
+      named_bar_sync(1, kSoft);
+      float m = -INFINITY, l = 0.f;
+      if (wg < 2) {
+        float2 o[kWg];
+#pragma unroll
+        for (int q = 0; q < kWg; ++q) {
+          o[q] = mrg[(q * 2 + wg) * BM + r];
+          m = fmaxf(m, o[q].x);
+        }
+        // an empty part has sum 0 (or NaN when its keys were all masked)
+#pragma unroll
+        for (int q = 0; q < kWg; ++q)
+          if (o[q].y > 0.f) l += o[q].y * ex2(o[q].x - m);
+      }
+      ok = named_bar_and(1, kSoft, ok);   // all read: the next piece may overwrite the area
       if (!ok) break;
-      const float m_own = w ? mh[1] : mh[0], l_own = w ? lh[1] : lh[0];
-      const float m = fmaxf(m_own, o.x);
-      // an empty half has sum 0 (or NaN when its keys were all masked)
-      const float l = (l_own > 0.f ? l_own * ex2(m_own - m) : 0.f) + (o.y > 0.f ? o.y * ex2(o.x - m) : 0.f);
-      p.ws_ml[((int64_t)x.u * p.maxp + x.k) * (2 * BM) + w * BM + r] = make_float2(m, l);
+      if (wg < 2) p.ws_ml[((int64_t)x.u * p.maxp + x.k) * (2 * BM) + wg * BM + r] = make_float2(m, l);
     }
   }
 
@@ -353,7 +363,6 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
   float* nlse = reinterpret_cast<float*>(sbase + kB_OffLse);
-  float* cs_b = reinterpret_cast<float*>(sbase + kB_OffCs);
   uint8_t* misc = sbase + kB_OffBar + B_NUM * 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
@@ -366,8 +375,8 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_NUM; ++i) {
       uint32_t cnt = 1;
-      if (i == B_ST_EMPTY || i == B_P_FULL || i == B_O_EMPTY) cnt = 256;   // both warpgroups
-      if (i == B_CS_FULL || i == B_CS_EMPTY) cnt = 128;                     // one warpgroup
+      if (i == B_P_FULL || i == B_O_EMPTY) cnt = kSoft;                  // every softmax thread
+      if (i == B_ST_EMPTY || i == B_ST_EMPTY + 1) cnt = kSoft / 2;        // one head's warpgroups
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -451,8 +460,8 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   } else if (warp == 1) {
     // =========================================================== MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_kk = idesc_bf16(128, 256, 0, 0);   // both operands K-major
-      const uint32_t idesc_mn = idesc_bf16(128, 256, 1, 1);   // both operands MN-major
+      const uint32_t idesc_st = idesc_bf16(128, 128, 0, 0);   // S^T of one head: K-major operands
+      const uint32_t idesc_mn = idesc_bf16(128, 256, 1, 1);   // O^T: both operands MN-major
       const uint32_t q_addr = base + kB_OffQ;
       const uint32_t p_addr = base + kB_OffP;
       bool ok = true;
@@ -464,23 +473,24 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         piece_tiles(x, g, t_lo, n);
         ok = mbar_wait(bar(B_Q), (uint32_t)pi & 1u, abort_flag, p.err, kWaitLimitNs, kErrTimeout);
         auto issue_st = [&](int j) -> bool {
-          // TMEM columns 0-255 (S^T) must have been read by both warpgroups
-          bool w_ok = st == 0 || mbar_wait(bar(B_ST_EMPTY), (uint32_t)(st - 1) & 1u, abort_flag, p.err,
-                                           kWaitLimitNs, kErrTimeout);
           const int pos = gp_base + k_pos(j), slot = pos % NS2;
-          if (w_ok)
-            w_ok = mbar_wait(bar(B_R_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, p.err,
-                             kWaitLimitNs, kErrTimeout);
-          if (!w_ok) return false;
-          tc_fence_after();
+          if (!mbar_wait(bar(B_R_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, p.err, kWaitLimitNs,
+                         kErrTimeout))
+            return false;
           const uint32_t k_addr = base + kB_OffR + (uint32_t)slot * kTile;
+          for (int hh = 0; hh < 2; ++hh) {
+            // head hh's S^T buffer must have been read by its two warpgroups
+            if (st > 0 && !mbar_wait(bar(B_ST_EMPTY + hh), (uint32_t)(st - 1) & 1u, abort_flag, p.err,
+                                     kWaitLimitNs, kErrTimeout))
+              return false;
+            tc_fence_after();
+            const uint32_t a0 = desc_lo(k_addr, 16), b0 = desc_lo(q_addr + (uint32_t)hh * 16384u, 16);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t da = smem_desc_sw128(k_addr + kmajor_off(kk, 128), 16, 1024);
-            const uint64_t db = smem_desc_sw128(q_addr + kmajor_off(kk, 256), 16, 1024);
-            umma_bf16(tmem, da, db, idesc_kk, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_bf16(tmem + (uint32_t)hh * 128u, a0 + (kmajor_off(kk, 128) >> 4), kDescHi,
+                        b0 + (kmajor_off(kk, 256) >> 4), kDescHi, idesc_st, kk > 0 ? 1u : 0u);
+            umma_commit(bar(B_ST_FULL + hh));
           }
-          umma_commit(bar(B_ST_FULL));
           umma_commit(bar(B_R_EMPTY + slot));
           ++st;
           return true;
@@ -499,13 +509,11 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                              kWaitLimitNs, kErrTimeout);
           if (!w_ok) return false;
           tc_fence_after();
-          const uint32_t v_addr = base + kB_OffR + (uint32_t)slot * kTile;
+          const uint32_t a0 = desc_lo(base + kB_OffR + (uint32_t)slot * kTile, kAtom), b0 = desc_lo(p_addr, kAtom);
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t da = smem_desc_sw128(v_addr + (uint32_t)kk * 2048u, kAtom, 1024);
-            const uint64_t db = smem_desc_sw128(p_addr + (uint32_t)kk * 2048u, kAtom, 1024);
-            umma_bf16(tmem + 256u, da, db, idesc_mn, (j > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_bf16(tmem + 256u, a0 + (uint32_t)kk * 128u, kDescHi, b0 + (uint32_t)kk * 128u, kDescHi, idesc_mn,
+                      (j > 0 || kk > 0) ? 1u : 0u);
           umma_commit(bar(B_P_EMPTY));
           umma_commit(bar(B_R_EMPTY + slot));
           ++ot;
@@ -526,23 +534,24 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   } else {
     // =========================================================== softmax / epilogue
-    const int w = (warp - 2) >> 2;                    // 0: head A, 1: head B
+    // Four warpgroups: warpgroup wg takes the 64 query columns [64 wg, 64 wg + 64)
+    // of S^T, i.e. queries [64 hq, 64 hq + 64) of head w (w = wg / 2, hq = wg % 2),
+    // and writes its own partial row of column sums.
+    const int wg = (warp - 2) >> 2;
+    const int w = wg >> 1, hq = wg & 1;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                 // TMEM lane: key in S^T, d in O^T
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t st_tmem = lane_base + (uint32_t)w * 128u;
-    const uint32_t o_tmem = lane_base + 256u + (uint32_t)w * 128u;
-    const uint32_t p_row = base + kB_OffP + (uint32_t)(2 * w) * kAtom + (uint32_t)(r >> 3) * 1024u +
+    const uint32_t st_tmem = lane_base + (uint32_t)wg * 64u;
+    const uint32_t o_tmem = lane_base + 256u + (uint32_t)wg * 64u;
+    const uint32_t p_row = base + kB_OffP + (uint32_t)wg * kAtom + (uint32_t)(r >> 3) * 1024u +
                            (uint32_t)(r & 7) * 128u;
-    const float* nl_w = nlse + w * BM;
+    const float* nl_w = nlse + wg * 64;
     const int64_t S = p.S, M = p.M, nv = p.n_valid;
     const float c = p.scale_log2;
-    const int t = threadIdx.x - 64;                    // 0..255 over both warpgroups
+    const int t = threadIdx.x - 64;                    // 0 .. kSoft-1 over all warpgroups
     bool ok = true;
     int st = 0;
-    float prev_cs = 0.f;                               // warpgroup 0: last tile's head-A sum,
-    float* prev_part = nullptr;                        // waiting for head B's
-    int64_t prev_col = -1;
     // every warp passes every named barrier below whatever its `ok`, so a warp
     // that aborted cannot leave the others waiting; only the work is skipped
     for (int pi = 0; pi < npc; ++pi) {
@@ -551,10 +560,10 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       int t_lo, n;
       piece_tiles(x, g, t_lo, n);
       const bool head_ok = w == 0 || g.has_b;
-      // the unit's log-sum-exp of row r of head w: its pieces' (max, sum) in piece order
-      named_bar_sync(1 + w, 128);                      // the previous piece is done with nlse
-      if (ok) {
-        const float2* ml = p.ws_ml + (int64_t)x.u * p.maxp * (2 * BM) + w * BM + r;
+      // the unit's log-sum-exp of row r of head wg (wg < 2): its pieces' (max, sum) in piece order
+      named_bar_sync(1, kSoft);                        // the previous piece is done with nlse
+      if (ok && wg < 2) {
+        const float2* ml = p.ws_ml + (int64_t)x.u * p.maxp * (2 * BM) + wg * BM + r;
         float mx = -INFINITY;
         for (int k = 0; k < x.np; ++k) {
           const float2 v = ml[(int64_t)k * (2 * BM)];
@@ -566,85 +575,57 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           if (v.y > 0.f) lsum += v.y * ex2(v.x - mx);
         }
         const int64_t row_i = g.i0 + r;
-        nlse[w * BM + r] = (head_ok && row_i < S && lsum > 0.f) ? -(mx + lg2(lsum)) : -INFINITY;
+        const bool row_head_ok = wg == 0 || g.has_b;
+        nlse[wg * BM + r] = (row_head_ok && row_i < S && lsum > 0.f) ? -(mx + lg2(lsum)) : -INFINITY;
       }
-      named_bar_sync(1 + w, 128);
-      float* part = p.partials + ((int64_t)g.bh * (p.n_pg * p.n_rt) + (g.pg * p.n_rt + g.rt)) * p.stride;
+      named_bar_sync(1, kSoft);
+      float* part = p.partials + ((int64_t)g.bh * (p.n_grp * p.n_rt) + ((g.pg * kStreamRows + wg) * p.n_rt + g.rt)) * p.stride;
       for (int j = 0; ok && j < n; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ST_FULL), (uint32_t)st & 1u, abort_flag, p.err,
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ST_FULL + w), (uint32_t)st & 1u, abort_flag, p.err,
                                                kWaitLimitNs, kErrTimeout));
         if (!ok) break;
         tc_fence_after();
-        if (w == 0 && st > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_FULL), (uint32_t)(st - 1) & 1u, abort_flag,
-                                                 p.err, kWaitLimitNs, kErrTimeout));
-          if (!ok) break;
-          const float other = cs_b[r];
-          mbar_arrive(bar(B_CS_EMPTY));
-          if (prev_col >= 0) prev_part[prev_col] = prev_cs + other;
-        }
         const int jg = t_lo + j;
         const bool cache = jg < g.nct;
         const int64_t key = cache ? (int64_t)jg * BN + r : (int64_t)(jg - g.nct) * BN + r;
         const bool key_ok = cache ? key < nv : key < S;
         // chunk key `key` is seen by query columns q with i0 + q >= key
-        const int qmin = cache ? 0 : (int)(key - g.i0 > 0 ? key - g.i0 : 0);
-        const bool full = __all_sync(0xffffffffu, key_ok && qmin == 0);
+        const int qmin = (cache ? 0 : (int)(key - g.i0 > 0 ? key - g.i0 : 0)) - 64 * hq;
+        const bool full = __all_sync(0xffffffffu, key_ok && qmin <= 0);
         uint64_t cs4[4] = {0ull, 0ull, 0ull, 0ull};
-        // both halves of the key's P^T row in registers before waiting for the
-        // buffer, so the previous tile's O^T MMA overlaps all the exponentials
-        uint32_t pk[32], pk2[32];
-        {
-          uint32_t v[2][32];
-          tmem_ld32(st_tmem, v[0]);
-          tmem_ld32(st_tmem + 32, v[1]);
-          tmem_wait_ld();
-          if (full) key_half<true>(v, nl_w, c, key_ok, qmin, cs4, pk);
-          else key_half<false>(v, nl_w, c, key_ok, qmin, cs4, pk);
-        }
-        // the second half in two 32-query pieces: fewer registers live beside
-        // the packed first half
+        // the key's 64 probabilities in registers before waiting for the P^T
+        // buffer, so the previous tile's O^T MMA overlaps the exponentials
+        uint32_t pk[32];
 #pragma unroll
         for (int qc = 0; qc < 2; ++qc) {
           uint32_t v[32];
-          tmem_ld32(st_tmem + 64 + qc * 32, v);
+          tmem_ld32(st_tmem + qc * 32, v);
           tmem_wait_ld();
           if (qc == 1) {
             tc_fence_before();
-            mbar_arrive(bar(B_ST_EMPTY));
+            mbar_arrive(bar(B_ST_EMPTY + w));
           }
-          if (full) key_part<true, 32>(v, nl_w + 64 + qc * 32, c, key_ok, qmin - 64 - qc * 32, cs4, pk2 + qc * 16);
-          else key_part<false, 32>(v, nl_w + 64 + qc * 32, c, key_ok, qmin - 64 - qc * 32, cs4, pk2 + qc * 16);
+          if (full) key_part<true, 32>(v, nl_w + qc * 32, c, key_ok, qmin - qc * 32, cs4, pk + qc * 16);
+          else key_part<false, 32>(v, nl_w + qc * 32, c, key_ok, qmin - qc * 32, cs4, pk + qc * 16);
         }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)st & 1u) ^ 1u, abort_flag,
                                                p.err, kWaitLimitNs, kErrTimeout));
         if (!ok) break;
         store_p_half(p_row, r, pk);
-        store_p_half(p_row + kAtom, r, pk2);
         fence_async_smem();
         mbar_arrive(bar(B_P_FULL));
-        const float cs = cs_total(cs4);
-        if (w == 0) {
-          prev_cs = cs;
-          prev_part = part;
-          prev_col = key_ok ? (cache ? key : M + key) : -1;
-        } else {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_EMPTY), ((uint32_t)st & 1u) ^ 1u, abort_flag,
-                                                 p.err, kWaitLimitNs, kErrTimeout));
-          if (!ok) break;
-          cs_b[r] = head_ok ? cs : 0.f;                // without a head B every p is 0
-          mbar_arrive(bar(B_CS_FULL));
-        }
+        // without a head B every p of warpgroups 2 and 3 is 0
+        if (key_ok) part[cache ? key : M + key] = head_ok ? cs_total(cs4) : 0.f;
         ++st;
       }
-      // ----- the piece's O^T (lane = d, columns = head w's 128 queries)
+      // ----- the piece's O^T (lane = d, columns = the warpgroup's 64 queries of head w)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), (uint32_t)pi & 1u, abort_flag, p.err,
                                                      kWaitLimitNs, kErrTimeout));
       if (ok) tc_fence_after();
-      const int gq = g.h * p.G + g.gl_a + w;           // query head of warpgroup w
-      float* wsp = p.ws_o + (((int64_t)x.u * p.maxp + x.k) * (2 * BM) + w * BM) * D;
+      const int gq = g.h * p.G + g.gl_a + w;           // query head of warpgroup wg
+      float* wsp = p.ws_o + (((int64_t)x.u * p.maxp + x.k) * (2 * BM) + wg * 64) * D;
 #pragma unroll 1
-      for (int ch = 0; ok && ch < 4; ++ch) {
+      for (int ch = 0; ok && ch < 2; ++ch) {
         uint32_t o[32];
         tmem_ld32(o_tmem + ch * 32, o);
         tmem_wait_ld();
@@ -653,7 +634,7 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + ((int64_t)g.b * p.Hq + gq) * S * D + r;
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
-              const int64_t qi = g.i0 + ch * 32 + k;
+              const int64_t qi = g.i0 + 64 * hq + ch * 32 + k;
               if (qi < S) dst[qi * D] = __float2bfloat16_rn(__uint_as_float(o[k]));
             }
           }
@@ -667,16 +648,17 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (x.np > 1 && p.out != nullptr) {
         // the last piece of the unit to get here adds all partials in piece order
         __threadfence();
-        named_bar_sync(3, 256);
+        named_bar_sync(3, kSoft);
         if (t == 0) *last_flag = atomicAdd(p.count + x.u, 1) == x.np - 1;
-        named_bar_sync(3, 256);
+        named_bar_sync(3, kSoft);
         if (*last_flag) {
           __threadfence();
           const float* ws0 = p.ws_o + (int64_t)x.u * p.maxp * (2 * BM) * D;
           // items (query q, 8 values of d from d0): four at a time, so that each
           // thread has 8 loads per piece in flight
           constexpr int kItems = 2 * BM * (D / 8);
-          for (int it0 = t; it0 < kItems; it0 += 4 * 256) {
+          static_assert(kItems % (4 * kSoft) == 0, "whole rounds of items");
+          for (int it0 = t; it0 < kItems; it0 += 4 * kSoft) {
             float4 lo[4], hi[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) lo[i] = hi[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -684,7 +666,7 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
               float4 a[4], b2[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                const int it = it0 + i * 256;
+                const int it = it0 + i * kSoft;
                 const float4* src = reinterpret_cast<const float4*>(
                     ws0 + ((int64_t)k * (2 * BM) + it / (D / 8)) * D + (it % (D / 8)) * 8);
                 a[i] = __ldcg(src);
@@ -698,7 +680,7 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const int it = it0 + i * 256;
+              const int it = it0 + i * kSoft;
               const int q = it / (D / 8), d0 = (it % (D / 8)) * 8;
               const int wq = q / BM;
               const int64_t qi = g.i0 + (q % BM);
@@ -717,12 +699,6 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           if (t == 0) p.count[x.u] = 0;
         }
       }
-    }
-    // the last tile's head-A column sums still wait for head B's
-    if (w == 0 && ok && st > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_FULL), (uint32_t)(st - 1) & 1u, abort_flag, p.err,
-                                             kWaitLimitNs, kErrTimeout));
-      if (ok && prev_col >= 0) prev_part[prev_col] = prev_cs + cs_b[r];
     }
   }
 
@@ -802,6 +778,7 @@ cudaError_t launch_attn_stream(const AttnArgs& a, const StreamPlan& pl, void* ws
   p.n_pg = (p.G + 1) / 2;
   p.n_rt = (int)((a.S + BM - 1) / BM);
   p.maxp = pl.maxp;
+  p.n_grp = stream_partial_groups(p.G);
   p.S = a.S;
   p.M = a.M;
   p.n_valid = a.n_valid;
@@ -824,7 +801,9 @@ cudaError_t launch_attn_stream(const AttnArgs& a, const StreamPlan& pl, void* ws
   cfg.attrs = at;
   cfg.numAttrs = 1;
   cfg.dynamicSmemBytes = kA_SmemBytes;
+  cfg.blockDim = dim3(kThreads);
   if ((e = cudaLaunchKernelEx(&cfg, lse_stream_kernel, mq, mk, mkc, p)) != cudaSuccess) return e;
+  cfg.blockDim = dim3(kThreads);
   at[0].val.programmaticStreamSerializationAllowed = 1;   // kernel B follows kernel A
   cfg.dynamicSmemBytes = kB_SmemBytes;
   return cudaLaunchKernelEx(&cfg, attn_stream_kernel, mq, mk, mv, mkc, mvc, p);

@@ -82,6 +82,7 @@ static_assert(2 * kSlot1 <= kRBytes, "sweep-1 slots fit in R");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;     // 1 s per wait
+constexpr uint32_t kDescHi = desc_hi_sw128(1024);   // 8 rows of 128 bytes between core-matrix groups
 
 enum { B_Q = 0, B_R1_FULL = 1, B_R1_EMPTY = 3, B_R2_FULL = 5, B_R2_EMPTY = B_R2_FULL + NS2,
        B_S_FULL = B_R2_EMPTY + NS2, B_S_EMPTY = B_S_FULL + 2, B_ST_FULL = B_S_EMPTY + 2,
@@ -271,12 +272,11 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                          kErrTimeout);
           if (!ok) break;
           tc_fence_after();
+          const uint32_t a0 = desc_lo(q_addr + (uint32_t)w * kAtom, 16), b0 = desc_lo(k_addr, 16);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t da = smem_desc_sw128(q_addr + (uint32_t)w * kAtom + kmajor_off(kk, 256), 16, 1024);
-            const uint64_t db = smem_desc_sw128(k_addr + kmajor_off(kk, 256), 16, 1024);
-            umma_bf16(tmem + (uint32_t)w * 256u, da, db, idesc_kk, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_bf16(tmem + (uint32_t)w * 256u, a0 + (kmajor_off(kk, 256) >> 4), kDescHi, b0 + (kmajor_off(kk, 256) >> 4),
+                      kDescHi, idesc_kk, kk > 0 ? 1u : 0u);
           umma_commit(bar(B_S_FULL + w));
         }
         if (ok) umma_commit(bar(B_R1_EMPTY + s));
@@ -293,13 +293,11 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                            kWaitLimitNs, kErrTimeout);
         if (!w_ok) return false;
         tc_fence_after();
-        const uint32_t k_addr = base + kOffR + (uint32_t)slot * kTile;
+        const uint32_t a0 = desc_lo(base + kOffR + (uint32_t)slot * kTile, 16), b0 = desc_lo(q_addr, 16);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t da = smem_desc_sw128(k_addr + kmajor_off(kk, 128), 16, 1024);
-          const uint64_t db = smem_desc_sw128(q_addr + kmajor_off(kk, 256), 16, 1024);
-          umma_bf16(tmem, da, db, idesc_kk, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(tmem, a0 + (kmajor_off(kk, 128) >> 4), kDescHi, b0 + (kmajor_off(kk, 256) >> 4), kDescHi, idesc_kk,
+                    kk > 0 ? 1u : 0u);
         umma_commit(bar(B_ST_FULL));
         umma_commit(bar(B_R2_EMPTY + slot));
         return true;
@@ -316,13 +314,11 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                            kWaitLimitNs, kErrTimeout);
         if (!w_ok) return false;
         tc_fence_after();
-        const uint32_t v_addr = base + kOffR + (uint32_t)slot * kTile;
+        const uint32_t a0 = desc_lo(base + kOffR + (uint32_t)slot * kTile, kAtom), b0 = desc_lo(p_addr, kAtom);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t da = smem_desc_sw128(v_addr + (uint32_t)kk * 2048u, kAtom, 1024);
-          const uint64_t db = smem_desc_sw128(p_addr + (uint32_t)kk * 2048u, kAtom, 1024);
-          umma_bf16(tmem + 256u, da, db, idesc_mn, (j > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16(tmem + 256u, a0 + (uint32_t)kk * 128u, kDescHi, b0 + (uint32_t)kk * 128u, kDescHi, idesc_mn,
+                    (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(B_P_EMPTY));
         umma_commit(bar(B_R2_EMPTY + slot));
         return true;

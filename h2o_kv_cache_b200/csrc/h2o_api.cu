@@ -255,14 +255,6 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   const int row_tile = decode ? (int)S : h->row_tile;
   const int n_rt = decode ? 1 : (int)((S + h->row_tile - 1) / h->row_tile);
   const int64_t stride = h2o::partial_stride(h->M, S);
-  const int n_grp = decode ? 1 : h2o::partial_groups(h->G, h->use_umma);
-  const size_t part_bytes = (size_t)BH * n_grp * n_rt * stride * sizeof(float);
-  H2O_CUDA(h, ensure(h->partials, part_bytes), "scratch alloc");
-  H2O_CUDA(h, ensure(h->freed, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
-  H2O_CUDA(h, ensure(h->evicted, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
-
-  cudaEvent_t* evs = h->ev[h->prof_steps % h2o_ctx::kProfRing];
-  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[0], st), "event");
 
   h2o::AttnArgs a;
   a.q = dq;
@@ -271,7 +263,6 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   a.out = dout;
   a.kc = h->kc;
   a.vc = h->vc;
-  a.partials = static_cast<float*>(h->partials.p);
   a.err = h->err;
   a.B = h->B;
   a.Hq = h->Hq;
@@ -284,6 +275,33 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   a.split = attn_split();
   a.inject_timeout = inject_timeout() ? 1 : 0;
   a.scale = (float)(1.0 / std::sqrt((double)h->d));
+
+  // tensor-core path: one kernel with both sweeps, or two kernels over a
+  // balanced partition of the key pairs ("stream").  Automatic: the partition
+  // pays when the one-kernel grid would leave SMs idle (n_sm / 2 .. 2 n_sm
+  // units) and units are long enough (>= 24 pairs on average) for a piece
+  // boundary's Q reload and epilogue.
+  h2o::StreamPlan pl;
+  bool stream = false;
+  if (!decode && h->use_umma) {
+    if (h->n_sm == 0) H2O_CUDA(h, cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device),
+                               "device attribute");
+    const int mode = attn_mode();
+    if (mode != 1 && !a.inject_timeout && h2o::attn_stream_plan(a, h->n_sm, &pl))
+      stream = mode == 2 || (2 * pl.units >= h->n_sm && pl.units <= 2 * h->n_sm &&
+                             pl.total_pairs >= 24 * (int64_t)pl.units);
+  }
+  const int n_grp = decode ? 1 : stream ? h2o::stream_partial_groups(h->G)
+                                        : h2o::partial_groups(h->G, h->use_umma);
+  const size_t part_bytes = (size_t)BH * n_grp * n_rt * stride * sizeof(float);
+  H2O_CUDA(h, ensure(h->partials, part_bytes), "scratch alloc");
+  a.partials = static_cast<float*>(h->partials.p);
+  H2O_CUDA(h, ensure(h->freed, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
+  H2O_CUDA(h, ensure(h->evicted, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
+
+  cudaEvent_t* evs = h->ev[h->prof_steps % h2o_ctx::kProfRing];
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[0], st), "event");
+
   if (fault_injected("launch")) return fail(h, H2O_ECUDA, "injected launch failure");
   cudaError_t e = cudaSuccess;
   int launches = 1;
@@ -309,17 +327,6 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
     da.scale_log2 = a.scale * 1.4426950408889634f;
     e = h2o::launch_decode(da, h->dtype, BH, true, st);
   } else if (h->use_umma) {
-    if (h->n_sm == 0) H2O_CUDA(h, cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device),
-                               "device attribute");
-    const int mode = attn_mode();
-    h2o::StreamPlan pl;
-    bool stream = false;
-    // automatic: a balanced partition pays when the one-kernel grid would
-    // leave SMs idle (n_sm / 2 .. 2 n_sm units) and units are long enough
-    // (>= 24 pairs on average) for a piece boundary's Q reload and epilogue
-    if (mode != 1 && !a.inject_timeout && h2o::attn_stream_plan(a, h->n_sm, &pl))
-      stream = mode == 2 || (2 * pl.units >= h->n_sm && pl.units <= 2 * h->n_sm &&
-                             pl.total_pairs >= 24 * (int64_t)pl.units);
     if (stream) {
       H2O_CUDA(h, ensure(h->ws_ml, pl.ml_bytes), "scratch alloc");
       if (pl.o_bytes) H2O_CUDA(h, ensure(h->ws_o, pl.o_bytes), "scratch alloc");

@@ -29,6 +29,10 @@ enum : int {
 // columns of keys it can see (key j < min(S, (rt + 1) * row_tile)).
 inline int64_t partial_stride(int64_t M, int64_t S) { return (M + S + 3) & ~(int64_t)3; }
 inline int partial_groups(int G, bool umma) { return umma ? (G + 1) / 2 : G; }
+// The stream-partitioned tensor-core path writes one partial row per softmax
+// warpgroup: kStreamRows per head pair (its four 64-query slices).
+constexpr int kStreamRows = 4;
+inline int stream_partial_groups(int G) { return kStreamRows * ((G + 1) / 2); }
 
 // Order in which a column's partial rows are added, shared by both tail paths
 // so they agree bit for bit: the column's list of n rows (for a chunk column,
