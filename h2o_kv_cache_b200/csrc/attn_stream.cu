@@ -66,6 +66,7 @@ constexpr uint32_t kB_OffBar = kB_OffLse + 2 * BM * 4;
 // so the softmax reads one head's tile while the other head's MMA runs
 enum { B_Q = 0, B_Q_EMPTY, B_R_FULL, B_R_EMPTY = B_R_FULL + NS2, B_ST_FULL = B_R_EMPTY + NS2,
        B_ST_EMPTY = B_ST_FULL + 2, B_P_FULL = B_ST_EMPTY + 2, B_P_EMPTY, B_O_FULL, B_O_EMPTY, B_DRAIN,
+       B_NEVER,   // test hook: nothing ever arrives on it
        B_NUM };
 
 // after the barriers: TMEM address, abort flag, the CTA's pieces
@@ -88,6 +89,7 @@ struct SParams {
   int* count;           // [units]: pieces of the unit done with sweep 2
   int B, Hq, Hkv, G, n_pg, n_rt, maxp;
   int n_grp;            // partial rows per (b, KV head, row tile): kStreamRows per head pair
+  int inject_timeout;   // test hook: one wait of kernel B runs out
   int64_t S, M, n_valid, stride;
   int64_t total_pairs;  // over all units
   float scale_log2;
@@ -552,6 +554,11 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int t = threadIdx.x - 64;                    // 0 .. kSoft-1 over all warpgroups
     bool ok = true;
     int st = 0;
+    if (p.inject_timeout && wg == 0) {
+      // test hook: a bounded wait on a barrier nothing completes runs out (1 ms);
+      // every role then leaves through its abort path and the step reports it
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_NEVER), 0, abort_flag, p.err, 1000000ull, kErrTimeout));
+    }
     // every warp passes every named barrier below whatever its `ok`, so a warp
     // that aborted cannot leave the others waiting; only the work is skipped
     for (int pi = 0; pi < npc; ++pi) {
@@ -779,6 +786,7 @@ cudaError_t launch_attn_stream(const AttnArgs& a, const StreamPlan& pl, void* ws
   p.n_rt = (int)((a.S + BM - 1) / BM);
   p.maxp = pl.maxp;
   p.n_grp = stream_partial_groups(p.G);
+  p.inject_timeout = a.inject_timeout;
   p.S = a.S;
   p.M = a.M;
   p.n_valid = a.n_valid;

@@ -155,7 +155,8 @@ int attn_mode() {
   return 0;
 }
 
-// H2O_INJECT_TIMEOUT=1 (test hook): in the tensor-core attention kernel one
+// H2O_INJECT_TIMEOUT=1 (test hook): in the tensor-core attention kernel (the
+// one-kernel path, or with H2O_ATTN_MODE=stream the second stream kernel) one
 // softmax warpgroup waits on a barrier that nothing completes, with a 1 ms
 // limit; the step then fails with H2O_ETIMEOUT and the context stays usable.
 bool inject_timeout() {
@@ -287,7 +288,7 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
     if (h->n_sm == 0) H2O_CUDA(h, cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device),
                                "device attribute");
     const int mode = attn_mode();
-    if (mode != 1 && !a.inject_timeout && h2o::attn_stream_plan(a, h->n_sm, &pl))
+    if (mode != 1 && (!a.inject_timeout || mode == 2) && h2o::attn_stream_plan(a, h->n_sm, &pl))
       stream = mode == 2 || (2 * pl.units >= h->n_sm && pl.units <= 2 * h->n_sm &&
                              pl.total_pairs >= 24 * (int64_t)pl.units);
   }

@@ -284,11 +284,14 @@ def test_shape_error_leaves_state_intact(h2o):
     cache.close()
 
 
-def test_bounded_wait_timeout_is_reported_and_context_stays_usable(h2o, monkeypatch):
+@pytest.mark.parametrize("mode", ["fused", "stream"])
+def test_bounded_wait_timeout_is_reported_and_context_stays_usable(h2o, monkeypatch, mode):
     # a wait on a barrier that nothing completes runs out (1 ms); every role of the
     # kernel leaves through its abort path, the step reports H2O_ETIMEOUT, and the
-    # device context keeps working
+    # device context keeps working.  "stream": the hook sits in the second of the
+    # two stream-partitioned kernels (four softmax warpgroups, per-piece barriers).
     from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    monkeypatch.setenv("H2O_ATTN_MODE", mode)
     cfg = _cfg(0, dtype=torch.bfloat16, d=128)
     Q, K, V = gen_batch(cfg, 0, device="cuda")
     chunks = split_chunks(Q, K, V, cfg.bounds())
