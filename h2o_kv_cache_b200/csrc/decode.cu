@@ -335,12 +335,19 @@ cudaError_t launch_dec_rows(const DecodeArgs& a, int BH, bool pdl, cudaStream_t 
 
 }  // namespace
 
-bool decode_supported(int G, int64_t S) { return S >= 1 && G * S <= 16; }
+// G * S <= 16 rows, and the scores of a CTA's keys fit its 160 KB with a
+// portable cluster of 8 CTAs (16-row chunks up to 20480 keys, 4-row ones up to
+// 81920); longer caches take the tensor-core path.
+bool decode_supported(int G, int64_t S, int64_t keys) {
+  if (S < 1 || G * S > 16) return false;
+  const int RM = G * S <= 4 ? 4 : 16;
+  return (keys + 7) / 8 * RM * 4 <= 160 * 1024;
+}
 
 // Keys per CTA and cluster size: at least 64 keys a CTA, scores within 160 KB
 // of shared memory, and every (b, KV head) cluster in one wave if possible.
 cudaError_t launch_decode(DecodeArgs a, int dtype, int BH, bool pdl, cudaStream_t st) {
-  if (!decode_supported(a.G, a.S) || (a.d != 64 && a.d != 128) || BH < 1) return cudaErrorInvalidValue;
+  if (!decode_supported(a.G, a.S, a.n_valid + a.S) || (a.d != 64 && a.d != 128) || BH < 1) return cudaErrorInvalidValue;
   const int RM = a.G * a.S <= 4 ? 4 : 16;
   const int64_t keys = a.n_valid + a.S;
   int kc = 1;

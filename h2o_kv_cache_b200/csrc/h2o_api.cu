@@ -248,10 +248,11 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
     dout = h->st_out.p;
   }
 
-  // chunks of a few tokens (G * S <= 16 rows per KV head) take the decode
-  // kernel, which writes one partial row per KV head; forcing a tensor-core
-  // path (H2O_ATTN_MODE) bypasses it
-  const bool decode = h2o::decode_supported(h->G, S) && attn_mode() == 0;
+  // chunks of a few tokens (G * S <= 16 rows per KV head, and a cache whose
+  // scores fit the decode kernel's shared memory) take the decode kernel, which
+  // writes one partial row per KV head; forcing a tensor-core path
+  // (H2O_ATTN_MODE) bypasses it
+  const bool decode = h2o::decode_supported(h->G, S, h->n_valid + S) && attn_mode() == 0;
   // scratch sized for this chunk
   const int row_tile = decode ? (int)S : h->row_tile;
   const int n_rt = decode ? 1 : (int)((S + h->row_tile - 1) / h->row_tile);

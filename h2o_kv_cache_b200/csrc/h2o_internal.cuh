@@ -141,7 +141,7 @@ struct DecodeArgs {
   int kc = 1;           // CTAs per cluster (set by launch_decode)
   int64_t per = 0;      // keys per CTA (set by launch_decode)
 };
-bool decode_supported(int G, int64_t S);
+bool decode_supported(int G, int64_t S, int64_t keys);
 cudaError_t launch_decode(DecodeArgs a, int dtype, int BH, bool pdl, cudaStream_t st);
 
 // Records msg as this thread's last error (h2o_last_error(NULL)); returns code.

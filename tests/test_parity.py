@@ -221,6 +221,10 @@ def test_decode_kernel_m2k_and_m32k(h2o):
     run_stream(h2o, cfg, heads=[(0, 0), (0, 7)], T=cfg.P + 40)
     cfg = _cfg(3, name="m32k-decode", S=1)
     run_stream(h2o, cfg, heads=[(0, 3)], T=cfg.P + 6, kv_check=False)
+    # 16 rows per KV head (S = 4, G = 4) on the 32k-slot cache: the scores do not
+    # fit the decode kernel's shared memory, so the step takes the tensor-core path
+    cfg = _cfg(3, name="m32k-s4", S=4)
+    run_stream(h2o, cfg, heads=[(0, 5)], T=cfg.P + 8, kv_check=False)
 
 
 def test_small_chunks_s128(h2o):
