@@ -21,6 +21,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -102,7 +103,7 @@ class ClockSampler:
         self.nvml = None
         self.result = None
         self.source = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"h2o_bench_clocks_gpu{index}.csv")
 
     def __enter__(self):
         try:
