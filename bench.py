@@ -349,7 +349,8 @@ def run_ours(args, cfg):
         # the events time the kernels, not the Python loop's launch latency
         # (reported as host_us_per_step).
         sleep_s = min(2.0, 1.5 * args.steps * host_us * 1e-6)
-        torch.cuda._sleep(int(sleep_s * 2.0e9))            # cycles at about the max SM clock
+        if hasattr(torch.cuda, "_sleep"):                  # a spin kernel (PyTorch's own)
+            torch.cuda._sleep(int(sleep_s * 2.0e9))        # cycles at about the max SM clock
         for i in range(args.steps):
             for cache, _ in layers:
                 cache.set_profiling(i % PROF_EVERY == 0, restart=False)
