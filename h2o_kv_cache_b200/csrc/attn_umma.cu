@@ -32,11 +32,14 @@
 // CTA goes to one partial row that a fixed-order reduction adds up.
 //
 // Warp roles (320 threads): warp 0 issues TMA loads (one thread), warp 1
-// allocates TMEM and issues the MMAs (one thread), warps 2-5 / 6-9 are the
-// softmax warpgroups of heads A / B (thread = TMEM lane).  TMEM: sweep 1 holds
-// S_A and S_B (256 columns each); sweep 2 holds S^T and O^T (256 each).  Every
-// mbarrier wait is bounded; a wait that runs out sets the kErrTimeout bit of
-// the device error word and all roles exit.
+// allocates TMEM and issues the MMAs (one thread), warps 2-5 / 6-9 are two
+// softmax warpgroups (thread = TMEM lane).  In sweep 1 both read each head's S
+// tile, warpgroup w taking keys [128 w, 128 w + 128) of it, and their (max,
+// sum) halves are merged once per unit; in sweep 2 warpgroup w takes head w's
+// query columns.  TMEM: sweep 1 holds S_A and S_B (256 columns each); sweep 2
+// holds S^T and O^T (256 each).  Every mbarrier wait is bounded; a wait that
+// runs out sets the kErrTimeout bit of the device error word and all roles
+// exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
