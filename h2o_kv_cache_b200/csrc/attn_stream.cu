@@ -20,8 +20,12 @@
 //            its fp32 partial O and the last piece to finish (an atomic count
 //            per unit) adds all of them in piece order and writes the output.
 // No CTA waits on another.  Both kernels use the pipelines of attn_umma.cu
-// (TMA producer warp, MMA warp, two softmax warpgroups), run back to back over
-// the CTA's pieces; every mbarrier wait is bounded.
+// (TMA producer warp, MMA warp), run back to back over the CTA's pieces, with
+// four softmax warpgroups: in kernel A each takes a quarter of every 256-key
+// tile's keys for both heads (the four (max, sum) are merged per piece); in
+// kernel B each takes 64 query columns of S^T, which is two 128-column
+// buffers, one per head, and writes its own partial row of column sums.
+// Every mbarrier wait is bounded.
 #include <cstdio>
 #include <vector>
 
