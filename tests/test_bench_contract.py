@@ -1,0 +1,70 @@
+"""bench.py's arithmetic and its reference arm, on the CPU.
+
+The roofline figures of the bench line rest on two counts: algorithmic FLOPs
+per attention launch (4 d per (query-head row, visible key) pair: QK^T and PV,
+the recompute of the second sweep not credited) and algorithmic bytes of score
+accumulate + select + scatter.  The FLOP counts are checked against the
+per-step figures derived independently for the measurement table of the
+workloads (42.96, 283.5, 1134 and 584 GFLOP for a full cache and one chunk),
+and the reference arm is run once to check its JSON line.
+"""
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("cid,gflop", [(1, 42.96), (2, 283.5), (3, 1134.0), (4, 584.0)])
+def test_flops_per_step_match_the_measurement_table(cid, gflop):
+    from h2o_kv_cache_b200.workload import CONFIGS
+    b = _bench()
+    cfg = CONFIGS[cid]
+    flops = 4 * cfg.d * b.attn_pairs(cfg, cfg.S, cfg.M)     # full cache, one chunk, one layer
+    assert abs(flops / 1e9 - gflop) / gflop < 1e-3, flops / 1e9
+
+
+def test_pairs_count_visible_keys():
+    # a brute count of (row, visible key) pairs on a small case
+    from h2o_kv_cache_b200.workload import Config
+    import torch
+    b = _bench()
+    cfg = Config(9, "t", 2, 6, 3, 16, 40, 4, 100, 40, 7, torch.float32, 0.0)
+    S, nv = 7, 40
+    brute = sum(nv + (i + 1) for _ in range(cfg.B * cfg.Hq) for i in range(S))
+    assert b.attn_pairs(cfg, S, nv) == brute
+
+
+def test_select_scatter_bytes():
+    from h2o_kv_cache_b200.workload import CONFIGS
+    b = _bench()
+    cfg = CONFIGS[1]
+    # scores and positions (4 B each) read and written for every slot, and the
+    # chunk's K and V rows (bf16) read and written, per (batch, KV head)
+    expect = cfg.B * cfg.Hkv * (cfg.M * 8 * 2 + cfg.S * cfg.d * 2 * 2 * 2)
+    assert b.select_scatter_bytes(cfg, cfg.S) == expect == 8650752
+
+
+def test_reference_arm_prints_one_json_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["metric"] == "H2O chunk-step query-tokens/s" and d["unit"] == "query-tokens/s"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
