@@ -3,15 +3,20 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
 One step = one chunk of S query tokens through the whole path (attention with
-summed weights, score accumulate, select, scatter) on one layer's caches.  The
-default workload is the 2k-slot / 1k-chunk configuration (B=1, Hq=32, Hkv=8,
-d=128, M=2048, R=256, bf16).  Inputs are resident in HBM before timing; L2 is
-flushed (a 256 MiB write) between steps, outside the per-step CUDA events.  At
-N > 1 GPUs every rank runs an independent replica on its own seeded stream (the
-path has no cross-GPU exchange); the time is the max over ranks.
+summed weights, score accumulate, select, scatter) on every layer's caches.  The
+default workload is the largest single-GPU one: B=4 sequences, 28 independent
+layer caches (Hq=32, Hkv=8, d=128, M=8192, R=512, bf16), chunks of S=1024; a step
+runs the chunk through all 28 layers.  The 16k-slot / 1k-chunk and 32k-slot /
+2k-chunk single-layer workloads are measured in the same run and reported under
+"other_workloads" (their attention and select/scatter roofline figures).
+Inputs are resident in HBM before timing; L2 is flushed (a 256 MiB write)
+between steps, outside the per-step CUDA events.  At N > 1 GPUs every rank runs
+an independent replica on its own seeded stream (the path has no cross-GPU
+exchange); the time is the max over ranks.
 
 Prints ONE JSON line (rank 0).  `--impl reference` times the float64 CPU oracle
-instead, on a bounded sample of the same workload (rank 0 only).
+instead, on a bounded sample of the same workload (rank 0 only); it loads no
+part of the CUDA library.
 """
 from __future__ import annotations
 
@@ -33,6 +38,33 @@ METRIC = "H2O chunk-step query-tokens/s"
 PROF_EVERY = 8     # timed steps per step with per-kernel events
 UNIT = "query-tokens/s"
 L2_FLUSH_BYTES = 256 << 20
+
+
+def workload_module():
+    """The seeded input generator, loaded from its file: importing it through the
+    package would load libh2o.so, which the reference arm must not map."""
+    import importlib.util
+    name = "h2o_bench_workload"
+    if name in sys.modules:
+        return sys.modules[name]
+    spec = importlib.util.spec_from_file_location(
+        name, os.path.join(ROOT, "h2o_kv_cache_b200", "workload.py"))
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[name] = mod
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def config_dict(cfg, world):
+    """The `config` object of the JSON line; both arms print the same one."""
+    return {"workload": f"{cfg.name}: {cfg.describe()}", "global_batch": cfg.B * world,
+            "seq_len": cfg.S, "layers": cfg.layers,
+            "parallelism": f"replicas x{world}" if world > 1 else "single",
+            "l2": "flushed between steps (256 MiB write outside the per-step events)"}
+
+
+def host_cores():
+    return {"blas_threads": blas_threads(), "os_cpu_count": os.cpu_count()}
 
 
 def load_peaks():
@@ -246,77 +278,103 @@ def oracle_sample(cfg, chunks_host, budget_s, max_head_chunks=None):
 
 
 def run_reference(args, cfg):
-    """--impl reference: the oracle as it stands, one (KV head, chunk) per step."""
+    """--impl reference: the oracle as it stands.  Each timed step is one
+    (batch 0, layer 0, KV head 0) cache taking one chunk; ms_per_step is that
+    measured time, and `value` extrapolates it to the whole workload step (all
+    batch x layer x KV head caches, which the oracle would run one after the
+    other).  Only rank 0 works; no part of the CUDA library is loaded."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
-    import numpy as np
-    n_needed = args.warmup + args.steps
-    T = min(cfg.T, cfg.P + cfg.S * max(1, min(n_needed, cfg.n_chunks)))
-    Q, K, V = gen_batch(cfg, 0, device="cpu", T=T)
-    ch = [tuple(x.double().numpy() for x in c)
-          for c in split_chunks(Q[:1], K[:1], V[:1], [(a, b) for a, b in cfg.bounds() if a < T])]
+    wl = workload_module()
     from oracle import H2OHeadOracle
+    n_needed = args.warmup + args.steps
+    n_ch = max(1, min(n_needed, cfg.n_chunks))
+    T = min(cfg.T, cfg.P + cfg.S * n_ch)
+    Q, K, V = wl.gen_sequence(cfg, 0, 0, device="cpu", T=T)
     G = cfg.G
+    q_all, k_all, v_all = (x[:G] if x is Q else x[:1] for x in (Q, K, V))
+    bounds = [(a, b) for a, b in cfg.bounds() if a < T]
+    ch = [(q_all[:, a:b].double().numpy(), k_all[0, a:b].double().numpy(), v_all[0, a:b].double().numpy())
+          for a, b in bounds]
     st = H2OHeadOracle(cfg.M, cfg.R, G, cfg.d)
-    q0, k0, v0 = ch[0]
-    st.step(q0[0, 0:G], k0[0, 0], v0[0, 0])
+    st.step(*ch[0])                                                      # prefill, untimed
     times = []
     for i in range(n_needed):
         q, k, v = ch[1 + i % (len(ch) - 1)]
         t = time.perf_counter()
-        st.step(q[0, 0:G], k[0, 0], v[0, 0])
+        st.step(q, k, v)
         dt = time.perf_counter() - t
         if i >= args.warmup:
             times.append(dt)
-    per_step = statistics.mean(times) * cfg.B * cfg.Hkv * cfg.layers
-    value = cfg.B * cfg.S / per_step
-    cores = blas_threads()
-    sample = (f"each step: the float64 oracle on one (batch 0, KV head 0) cache for one chunk, "
-              f"scaled x{cfg.B * cfg.Hkv * cfg.layers} (batch, layer, KV head) caches to a whole step")
+    per_head_s = statistics.mean(times)
+    caches = cfg.B * cfg.Hkv * cfg.layers
+    value = cfg.B * cfg.S / (per_head_s * caches)
+    cores = host_cores()
+    sample = (f"each timed step: the float64 oracle on one (batch 0, layer 0, KV head 0) cache taking "
+              f"one chunk; value extrapolates x{caches} (batch, layer, KV head) caches to a whole step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_head_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": {"workload": f"{cfg.name}: {cfg.describe()}", "parallelism": "replicas"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": sample},
+            "data": "synthetic", "config": config_dict(cfg, world),
+            "extrapolation": {"caches_per_workload_step": caches,
+                              "ms_per_workload_step": per_head_s * caches * 1e3,
+                              "ms_per_step_is": "one (batch, layer, KV head) cache, measured"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores["blas_threads"],
+                             "os_cpu_count": cores["os_cpu_count"], "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, cfg):
-    world, rank, local = dist_setup(args.gpus)
+def traffic_for(cfg):
+    """DRAM bytes per attention launch from one ncu capture, while the sources
+    it was taken on are unchanged; None otherwise."""
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(tfile):
+        return None
+    try:
+        with open(tfile) as f:
+            ent = json.load(f).get(cfg.name)
+        if ent and ent.get("sources_sha") == sources_sha(KERNEL_SOURCES[ent["path"]]):
+            return ent["dram_bytes_per_launch"]
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
+def measure(args, cfg, world, rank, local, steps, with_e2e):
+    """Times `steps` steps of workload cfg on this rank's GPU; returns a dict of
+    figures (device-timed value, per-kernel times, roofline, e2e)."""
     import h2o_kv_cache_b200 as h2o
-    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    wl = workload_module()
     from h2o_kv_cache_b200.replicas import aggregate_throughput, replica_stream_layer
     dev = torch.device("cuda", local if world > 1 else 0)
-    n_needed = args.warmup + 2 * args.steps + 1     # device-timed steps, then host-buffer steps
+    n_needed = args.warmup + (2 if with_e2e else 1) * steps + 1
     n_chunks = min(cfg.n_chunks, n_needed)
     T = cfg.P + cfg.S * n_chunks
     bounds = [(a, b) for a, b in cfg.bounds() if a < T]
     layers = []                                    # per layer: (cache, chunks)
     for layer in range(cfg.layers):
         # each replica (rank) has its own seeded streams
-        Q, K, V = gen_batch(cfg, replica_stream_layer(rank, layer), device=dev, T=T)
-        chunks = split_chunks(Q, K, V, bounds)
+        Q, K, V = wl.gen_batch(cfg, replica_stream_layer(rank, layer), device=dev, T=T)
+        chunks = wl.split_chunks(Q, K, V, bounds)
         del Q, K, V
         cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype, device=dev)
         cache.prefill(*chunks[0], want_out=False)
         layers.append((cache, chunks))
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    out = torch.empty_like(layers[0][1][1][0])
+    outs = [torch.empty_like(layers[0][1][1][0]) for _ in layers]
     n_avail = len(bounds) - 1
     ci = 0
 
-    def step_all(out_buf, host=None):
+    def step_all(out_bufs, host=None):
         """One step: the next chunk through every layer's cache."""
         nonlocal ci
         for li, (cache, chunks) in enumerate(layers):
             c = host[li] if host is not None else chunks[1 + ci % n_avail]
-            cache.step(*c, out=out_buf)
+            cache.step(*c, out=out_bufs[li])
         ci += 1
 
     # warm-up; the host's enqueue time per step is measured on the last ones
@@ -325,7 +383,7 @@ def run_ours(args, cfg):
         torch.cuda.synchronize(dev)
         t = time.perf_counter()
         flush.zero_()
-        step_all(out)
+        step_all(outs)
         host_s.append(time.perf_counter() - t)
     torch.cuda.synchronize(dev)
     host_us = 1e6 * min(host_s[1:] if len(host_s) > 1 else host_s)
@@ -335,12 +393,12 @@ def run_ours(args, cfg):
     for cache, _ in layers:
         cache.set_profiling(True)       # restart the count of profiled steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+          for _ in range(steps)]
     kern_ms = []
     pairs = 0
     launches = 0
     barrier(world)
-    n_prof = (args.steps + PROF_EVERY - 1) // PROF_EVERY
+    n_prof = (steps + PROF_EVERY - 1) // PROF_EVERY
     if n_prof > 64:
         raise SystemExit(f"--steps must be <= {64 * PROF_EVERY} (per-kernel event ring)")
     with ClockSampler(local if world > 1 else 0) as clocks:
@@ -348,17 +406,17 @@ def run_ours(args, cfg):
         # region).  A GPU sleep outside every event lets the host get ahead, so
         # the events time the kernels, not the Python loop's launch latency
         # (reported as host_us_per_step).
-        sleep_s = min(2.0, 1.5 * args.steps * host_us * 1e-6)
+        sleep_s = min(2.0, 1.5 * steps * host_us * 1e-6)
         if hasattr(torch.cuda, "_sleep"):                  # a spin kernel (PyTorch's own)
             torch.cuda._sleep(int(sleep_s * 2.0e9))        # cycles at about the max SM clock
-        for i in range(args.steps):
+        for i in range(steps):
             for cache, _ in layers:
                 cache.set_profiling(i % PROF_EVERY == 0, restart=False)
             flush.zero_()
             for cache, _ in layers:
                 pairs += attn_pairs(cfg, cfg.S, cache.info()["n_valid"])
             ev[i][0].record(stream)
-            step_all(out)
+            step_all(outs)
             ev[i][1].record(stream)
             launches += sum(c.info()["launches"] for c, _ in layers)
         barrier(world)
@@ -369,85 +427,108 @@ def run_ours(args, cfg):
         kern_ms.append(t)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_s = max_over_ranks(sum(step_ms) / 1e3, world)
-    value = aggregate_throughput(cfg.B * cfg.S * args.steps, world, total_s)
+    value = aggregate_throughput(cfg.B * cfg.S * steps, world, total_s)
     attn_ms = statistics.mean(k[0] for k in kern_ms) / cfg.layers
     sel_ms = statistics.mean(k[1] for k in kern_ms) / cfg.layers
-
-    # end to end through the C ABI with host buffers (pinned), copies inside the region
     for cache, _ in layers:
         cache.set_profiling(False)
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = d2h = 0
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-    pinned = {}                                    # one pinned host copy per distinct chunk
-    host_steps = []
-    for i in range(args.steps):
-        j = 1 + (ci + i) % n_avail
-        if j not in pinned:
-            pinned[j] = [tuple(x.cpu().pin_memory() for x in chunks[j]) for _, chunks in layers]
-        host_steps.append(pinned[j])
-    h2d = sum(x.numel() * x.element_size() for hs in host_steps[0] for x in hs)
-    d2h = hout.numel() * hout.element_size() * len(layers)
-    barrier(world)
-    for i in range(args.steps):
-        flush.zero_()
-        e2e_ev[i][0].record(stream)
-        step_all(hout, host=host_steps[i])
-        e2e_ev[i][1].record(stream)
-    barrier(world)
-    e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3, world)
-    e2e_value = aggregate_throughput(cfg.B * cfg.S * args.steps, world, e2e_s)
 
-    peaks = load_peaks()
-    flops = 4 * cfg.d * pairs / (args.steps * cfg.layers)       # per attention launch
-    achieved_tflops = flops / (attn_ms * 1e-3) / 1e12
-    sel_bytes = select_scatter_bytes(cfg, cfg.S)
-    traffic = None
-    tfile = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tfile):
-        try:
-            with open(tfile) as f:
-                ent = json.load(f).get(cfg.name)
-            if ent and ent.get("sources_sha") == sources_sha(KERNEL_SOURCES[ent["path"]]):
-                traffic = ent["dram_bytes_per_launch"]
-        except (OSError, ValueError):
-            traffic = None
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_s * 1e3 / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32", "data": "synthetic",
-        "config": {"workload": f"{cfg.name}: {cfg.describe()}", "global_batch": cfg.B * world,
-                   "seq_len": cfg.S, "parallelism": f"replicas x{world}" if world > 1 else "single",
-                   "l2": "flushed between steps (256 MiB write outside the per-step events)",
-                   "kernel_events": f"CUDA events around each kernel on every {PROF_EVERY}th timed step"},
-        "roofline": {"bound": "tensor", "achieved": achieved_tflops,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved_tflops / peaks["bf16_tflops"], "traffic": traffic,
-                     "kernel": "attention + summed weights",
-                     "peak_source": f"{peaks['source']} bf16 dense (burst)",
-                     "algorithmic_flops_per_launch": flops, "ms_per_launch": attn_ms},
-        "roofline_select_scatter": {"bound": "hbm", "achieved": sel_bytes / (sel_ms * 1e-3) / 1e9,
-                                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                    "frac": sel_bytes / (sel_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                                    "algorithmic_bytes_per_launch_set": sel_bytes,
-                                    "ms_per_launch_set": sel_ms},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches,
-        "host_us_per_step": host_us,
-        "clocks": clocks.summary(),
-        "kernel_ms_per_layer": {"attention": attn_ms,
-                                "tail (score accumulate + select + scatter)": sel_ms},
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        chunks0 = layers[0][1]
-        chunks_host = [tuple(x[:1].double().cpu().numpy() for x in c) for c in chunks0[:8]]
-        rate, desc, n, el = oracle_sample(cfg, chunks_host, budget_s=args.cpu_budget)
-        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(),
-                                "kind": "oracle", "sample": desc}
+    res = {"value": value, "ms_per_step": total_s * 1e3 / steps, "steps": steps,
+           "launches": launches, "host_us": host_us, "clocks": clocks.summary(),
+           "attn_ms": attn_ms, "sel_ms": sel_ms,
+           "flops": 4 * cfg.d * pairs / (steps * cfg.layers)}          # per attention launch
+    if with_e2e:
+        # end to end through the C ABI with host buffers (pinned), copies inside the
+        # region: per layer one pinned (q, k, v) set per distinct chunk, at most two
+        # distinct chunks (the caches keep evolving whatever the values)
+        houts = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(steps)]
+        pinned = {}
+        host_steps = []
+        for i in range(steps):
+            j = 1 + (ci + i % 2) % n_avail
+            if j not in pinned:
+                pinned[j] = [tuple(x.cpu().pin_memory() for x in chunks[j]) for _, chunks in layers]
+            host_steps.append(pinned[j])
+        h2d = sum(x.numel() * x.element_size() for hs in host_steps[0] for x in hs)
+        d2h = sum(o.numel() * o.element_size() for o in houts)
+        barrier(world)
+        for i in range(steps):
+            flush.zero_()
+            e2e_ev[i][0].record(stream)
+            step_all(houts, host=host_steps[i])
+            e2e_ev[i][1].record(stream)
+        barrier(world)
+        e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3, world)
+        res["e2e"] = {"value": aggregate_throughput(cfg.B * cfg.S * steps, world, e2e_s),
+                      "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del pinned, host_steps, houts
+    if with_e2e:   # the chunks the oracle's CPU baseline is timed on
+        res["chunks0_host"] = [tuple(x[:1].double().cpu().numpy() for x in c) for c in layers[0][1][:8]]
     for cache, _ in layers:
         cache.close()
+    del layers, outs, flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def roofline_objects(cfg, res, peaks):
+    achieved = res["flops"] / (res["attn_ms"] * 1e-3) / 1e12
+    sel_bytes = select_scatter_bytes(cfg, cfg.S)
+    sel_gbs = sel_bytes / (res["sel_ms"] * 1e-3) / 1e9
+    return (
+        {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+         "frac": achieved / peaks["bf16_tflops"], "traffic": traffic_for(cfg),
+         "kernel": "attention + summed weights",
+         "peak_source": f"{peaks['source']} bf16 dense (burst)",
+         "algorithmic_flops_per_launch": res["flops"], "ms_per_launch": res["attn_ms"]},
+        {"bound": "hbm", "achieved": sel_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+         "frac": sel_gbs / peaks["hbm_gbs"], "kernel": "tail: score accumulate + select + scatter",
+         "peak_source": f"{peaks['source']} copy bandwidth",
+         "algorithmic_bytes_per_launch_set": sel_bytes, "ms_per_launch_set": res["sel_ms"]})
+
+
+def run_ours(args, cfg):
+    world, rank, local = dist_setup(args.gpus)
+    wl = workload_module()
+    peaks = load_peaks()
+    res = measure(args, cfg, world, rank, local, args.steps, with_e2e=True)
+    roof, roof_sel = roofline_objects(cfg, res, peaks)
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": config_dict(cfg, world),
+        "roofline": roof,
+        "roofline_select_scatter": roof_sel,
+        "e2e": res["e2e"],
+        "gpu_launches": res["launches"],
+        "host_us_per_step": res["host_us"],
+        "clocks": res["clocks"],
+        "kernel_ms_per_layer": {"attention": res["attn_ms"],
+                                "tail (score accumulate + select + scatter)": res["sel_ms"]},
+        "kernel_events": f"CUDA events around each kernel on every {PROF_EVERY}th timed step",
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, n, el = oracle_sample(cfg, res["chunks0_host"], budget_s=args.cpu_budget)
+        cores = host_cores()
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores["blas_threads"],
+                                "os_cpu_count": cores["os_cpu_count"], "kind": "oracle",
+                                "sample": desc}
+    # the other full-size single-layer workloads: their roofline figures
+    if not args.no_extra and args.config == 4:
+        other = {}
+        for cid in (2, 3):
+            c2 = wl.CONFIGS[cid]
+            r2 = measure(args, c2, world, rank, local, min(args.steps, 24), with_e2e=False)
+            ro, rs = roofline_objects(c2, r2, peaks)
+            other[c2.name] = {"workload": f"{c2.name}: {c2.describe()}", "value": r2["value"],
+                              "unit": UNIT, "steps": r2["steps"], "ms_per_step": r2["ms_per_step"],
+                              "roofline": ro, "roofline_select_scatter": rs,
+                              "gpu_launches": r2["launches"], "clocks": r2["clocks"]}
+        line["other_workloads"] = other
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -475,11 +556,13 @@ def sources_sha(names):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the 16k- and 32k-slot workloads measured after the default one")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--clock-poller", type=int, default=None, help=argparse.SUPPRESS)
     args = ap.parse_args()
@@ -488,8 +571,7 @@ def main():
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    from h2o_kv_cache_b200.workload import CONFIGS
-    cfg = CONFIGS[args.config]
+    cfg = workload_module().CONFIGS[args.config]
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

@@ -187,16 +187,62 @@ def attend_noalloc(q, k, v, k_cache, v_cache, n_valid: int, M: int, out=None, co
     no device memory itself (for callers that cannot call cudaMalloc).  Every
     buffer comes from the caller: q [B,Hq,S,d], k/v [B,Hkv,S,d], k_cache/v_cache
     [B,Hkv,M,d] (None when n_valid == 0), out [B,Hq,S,d], colsum [B,Hkv,M+S] f32.
-    Returns (out, colsum)."""
+    Returns (out, colsum).
+
+    The library reads and writes these buffers through raw pointers and cannot
+    check their sizes, so every shape, dtype, layout and device is checked here
+    first (ValueError), before any pointer crosses the C ABI."""
+    if not isinstance(q, torch.Tensor) or q.dtype not in _DTYPES:
+        raise ValueError("q must be a float32 or bfloat16 tensor")
+    if q.dim() != 4:
+        raise ValueError(f"q must be 4-d [B, Hq, S, d], got shape {tuple(q.shape)}")
     B, Hq, S, d = q.shape
+    dev = q.device
+
+    def _need(name, t, shape, dtype):
+        if not isinstance(t, torch.Tensor):
+            raise ValueError(f"{name} must be a tensor")
+        if t.dtype != dtype:
+            raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+        if t.device != dev:
+            raise ValueError(f"{name} must be on {dev}, got {t.device}")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+    _need("q", q, (B, Hq, S, d), q.dtype)
+    if k.dim() != 4:
+        raise ValueError(f"k must be 4-d [B, Hkv, S, d], got shape {tuple(k.shape)}")
     Hkv = k.shape[1]
-    dtype = _DTYPES[q.dtype]
+    if Hkv < 1 or Hq % Hkv != 0:
+        raise ValueError(f"Hq={Hq} must be a multiple of Hkv={Hkv}")
+    _need("k", k, (B, Hkv, S, d), q.dtype)
+    _need("v", v, (B, Hkv, S, d), q.dtype)
+    n_valid, M = int(n_valid), int(M)
+    if M < 1 or not 0 <= n_valid <= M:
+        raise ValueError(f"need M >= 1 and 0 <= n_valid <= M (n_valid={n_valid}, M={M})")
+    if n_valid > 0:
+        if k_cache is None or v_cache is None:
+            raise ValueError("k_cache and v_cache are required when n_valid > 0")
+        _need("k_cache", k_cache, (B, Hkv, M, d), q.dtype)
+        _need("v_cache", v_cache, (B, Hkv, M, d), q.dtype)
+    else:
+        for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+            if t is not None:
+                _need(name, t, (B, Hkv, M, d), q.dtype)
     if out is None:
         out = torch.empty_like(q)
+    else:
+        _need("out", out, (B, Hq, S, d), q.dtype)
     if colsum is None:
-        colsum = torch.empty(B, Hkv, M + S, dtype=torch.float32, device=q.device)
-    with torch.cuda.device(q.device):
+        colsum = torch.empty(B, Hkv, M + S, dtype=torch.float32, device=dev)
+    else:
+        _need("colsum", colsum, (B, Hkv, M + S), torch.float32)
+    if not q.is_cuda:
+        raise ValueError("every buffer must be a CUDA tensor")
+    with torch.cuda.device(dev):
         _check(lib.h2o_attend_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
-                                      B, Hq, Hkv, d, dtype, M, n_valid, S, _ptr(out), _ptr(colsum),
-                                      _stream_ptr(stream, q.device)))
+                                      B, Hq, Hkv, d, _DTYPES[q.dtype], M, n_valid, S, _ptr(out),
+                                      _ptr(colsum), _stream_ptr(stream, dev)))
     return out, colsum

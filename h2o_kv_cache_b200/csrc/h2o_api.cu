@@ -411,17 +411,41 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   return H2O_OK;
 }
 
-int alloc_state(h2o_ctx* h, int B) {
+// Frees the per-handle device state (cache, scores, positions, error word,
+// events); pointers are reset so the handle can be destroyed or prefilled again.
+void release_state(h2o_ctx* h) {
+  cudaFree(h->kc);
+  cudaFree(h->vc);
+  cudaFree(h->scores);
+  cudaFree(h->pos);
+  if (h->err) cudaFreeHost(h->err);
+  if (h->err_ev) cudaEventDestroy(h->err_ev);
+  for (auto& set : h->ev)
+    for (auto& ev : set) {
+      if (ev) cudaEventDestroy(ev);
+      ev = nullptr;
+    }
+  h->kc = h->vc = nullptr;
+  h->scores = nullptr;
+  h->pos = nullptr;
+  h->err = nullptr;
+  h->err_ev = nullptr;
+  h->device = -1;
+  cudaGetLastError();
+}
+
+int alloc_state_impl(h2o_ctx* h, int B) {
   const size_t es = elem_size(h->dtype);
   const size_t slots = (size_t)B * h->Hkv * h->M;
-  H2O_CUDA(h, cudaGetDevice(&h->device), "cudaGetDevice");
+  // the cache first: an injected allocation failure (H2O_FAULT=alloc) is
+  // reported before any other CUDA call
   H2O_CUDA(h, dev_alloc(&h->kc, slots * h->d * es), "cache alloc");
+  H2O_CUDA(h, cudaGetDevice(&h->device), "cudaGetDevice");
   H2O_CUDA(h, dev_alloc(&h->vc, slots * h->d * es), "cache alloc");
   H2O_CUDA(h, dev_alloc((void**)&h->scores, slots * sizeof(float)), "state alloc");
   H2O_CUDA(h, dev_alloc((void**)&h->pos, slots * sizeof(int32_t)), "state alloc");
   {
     void* hp = nullptr;
-    if (fault_injected("alloc")) return cuda_fail(h, cudaErrorMemoryAllocation, "state alloc");
     H2O_CUDA(h, cudaHostAlloc(&hp, sizeof(int), cudaHostAllocMapped), "pinned alloc");
     h->err = static_cast<int*>(hp);
     *h->err = 0;
@@ -436,6 +460,13 @@ int alloc_state(h2o_ctx* h, int B) {
   H2O_CUDA(h, cudaDeviceSynchronize(), "state init");
   h->B = B;
   return H2O_OK;
+}
+
+// On failure nothing stays allocated: the handle is as before the call.
+int alloc_state(h2o_ctx* h, int B) {
+  const int rc = alloc_state_impl(h, B);
+  if (rc != H2O_OK) release_state(h);
+  return rc;
 }
 
 }  // namespace
@@ -591,18 +622,10 @@ int h2o_destroy(h2o_t h) {
     cudaSetDevice(h->device);
     cudaDeviceSynchronize();
   }
-  cudaFree(h->kc);
-  cudaFree(h->vc);
-  cudaFree(h->scores);
-  cudaFree(h->pos);
-  if (h->err) cudaFreeHost(h->err);
   for (DevBuf* b : {&h->partials, &h->newscore, &h->freed, &h->evicted, &h->ws_ml, &h->ws_o,
                     &h->ws_count, &h->st_q, &h->st_k, &h->st_v, &h->st_out})
     cudaFree(b->p);
-  if (h->err_ev) cudaEventDestroy(h->err_ev);
-  for (auto& set : h->ev)
-    for (auto ev : set)
-      if (ev) cudaEventDestroy(ev);
+  release_state(h);
   delete h;
   return H2O_OK;
 }

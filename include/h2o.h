@@ -42,9 +42,18 @@
  *
  * Errors: every call returns an h2o_status; nothing aborts or throws across the
  * ABI.  h2o_last_error() gives the message of the last failing call.  A device
- * error raised by an earlier step (e.g. a bounded wait that timed out inside a
- * kernel) is reported by the next call on the handle as H2O_ETIMEOUT or
- * H2O_ECUDA.
+ * error raised inside a step's kernels (a bounded wait that timed out, too few
+ * evictable slots found on the device) is written to the handle's device error
+ * word and reported by a LATER call on the handle, as H2O_ETIMEOUT, H2O_ESHAPE
+ * or H2O_ECUDA: the first call that finds the step's work finished (steps do
+ * not wait for the GPU, so that may be several steps later).  Such a report
+ * does not name the step that failed, and every step enqueued since the last
+ * point at which the handle was known to be clean (a call that returned after
+ * waiting for the GPU: a step with host buffers, a read-back into host memory,
+ * or any step while the environment sets H2O_SYNC_CHECK=1) has then run on a
+ * cache whose contents are unspecified: destroy the handle.  With
+ * H2O_SYNC_CHECK=1 every step waits for its own kernels and reports its own
+ * device error.
  */
 #ifndef H2O_H_
 #define H2O_H_

@@ -3,8 +3,11 @@
 Tolerances (written here, used by every parity test):
   outputs  float32: |gpu - ref| <= 1e-4 * max_c |ref[..., c]| (each output row's
            largest component), elementwise
-           bfloat16: |gpu - ref| <= 2e-2 absolute (the relative norm error is also
-           reported)
+           bfloat16: |gpu - ref| <= 2e-2 absolute, and per (chunk, batch, KV head)
+           ||gpu - ref|| / ||ref|| <= 1e-2 (outputs of near-uniform attention over
+           thousands of keys are ~1e-2 in size, so the absolute bound alone would
+           pass a PV product that dropped a whole V tile; bf16 rounding of P and
+           of the output gives a relative norm error of a few 1e-3)
   scores   |gpu - ref| <= 1e-3 * |ref|
   evicted slots and slot -> position maps: bit-exact where the oracle's rank gap
   at the eviction boundary exceeds 1e-3; otherwise every slot in the symmetric
@@ -18,6 +21,7 @@ import torch
 
 OUT_RTOL_F32 = 1e-4
 OUT_ATOL_BF16 = 2e-2
+OUT_RELNORM_BF16 = 1e-2
 SCORE_RTOL = 1e-3
 GAP_TOL = 1e-3
 
@@ -37,10 +41,11 @@ def check_outputs(gpu, ref, dtype, where=""):
         bad = err > bound
         assert not bad.any(), (f"{where}: {int(bad.sum())} fp32 outputs out of tolerance, "
                                f"max err {err.max():.3e}")
-    else:
-        assert err.max() <= OUT_ATOL_BF16, f"{where}: bf16 output max err {err.max():.3e}"
     rel = float(np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-30))
-    return {"max_abs": float(err.max()), "rel_norm": rel}
+    if dtype != torch.float32:
+        assert err.max() <= OUT_ATOL_BF16, f"{where}: bf16 output max err {err.max():.3e}"
+        assert rel <= OUT_RELNORM_BF16, f"{where}: bf16 output relative norm error {rel:.3e}"
+    return {"max_abs": float(err.max()) if err.size else 0.0, "rel_norm": rel}
 
 
 def check_scores(gpu, ref, valid, where=""):
@@ -85,8 +90,27 @@ def check_evictions(head, gpu_freed, where=""):
         assert head.last_eligible[s], f"{where}: GPU evicted an ineligible slot {s}"
         assert abs(pre[s] - boundary) <= GAP_TOL * abs(boundary), (
             f"{where}: slot {s} score {pre[s]} is not within {GAP_TOL} of the boundary {boundary}")
-    assert got[:need].tolist() == sorted(got[:need].tolist()), f"{where}: evictions not ascending"
+    assert np.all(np.diff(got) > 0), f"{where}: filled slots not strictly ascending (duplicates?)"
     return "ties"
+
+
+def check_tie_state(gpu_freed, gpu_pos, pos_before, t0, where=""):
+    """Validity of a step whose eviction set the oracle does not fix (a near-tie):
+    the filled slots are unique and ascending, chunk token t0 + i sits in the
+    i-th filled slot, each new token appears exactly once, and every slot that was
+    not filled kept the position it held before the step."""
+    freed = np.asarray(gpu_freed)
+    pos = np.asarray(gpu_pos)
+    before = np.asarray(pos_before)
+    S = freed.size
+    assert np.all(np.diff(freed) > 0), f"{where}: filled slots not strictly ascending"
+    assert freed.min() >= 0 and freed.max() < pos.size, f"{where}: filled slot out of range"
+    assert np.array_equal(pos[freed], t0 + np.arange(S)), f"{where}: slot -> new token map wrong"
+    new = np.sort(pos[pos >= t0])
+    assert np.array_equal(new, t0 + np.arange(S)), f"{where}: new tokens not each cached once"
+    kept = np.ones(pos.size, bool)
+    kept[freed] = False
+    assert np.array_equal(pos[kept], before[kept]), f"{where}: a slot not filled changed position"
 
 
 def annotate_boundary(head, pos_before):

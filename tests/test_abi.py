@@ -89,3 +89,18 @@ def test_select_rejects_bad_sizes():
     assert _lib.lib.h2o_select(None, dummy, 1, 8, 10, 1, 2, dummy, None) == _lib.H2O_EINVAL
     # need == 0 is a no-op that touches no memory
     assert _lib.lib.h2o_select(dummy, dummy, 1, 8, 10, 1, 0, None, None) == _lib.H2O_OK
+
+
+def test_injected_allocation_failure_is_reported(monkeypatch):
+    # H2O_FAULT=alloc makes every device allocation of the library fail; it is
+    # made on the host, before any CUDA call, so no GPU is needed to see it
+    monkeypatch.setenv("H2O_FAULT", "alloc")
+    rc, h = _create()
+    assert rc == _lib.H2O_OK
+    dummy = ctypes.c_void_p(16)
+    assert _lib.lib.h2o_prefill(h, dummy, dummy, dummy, None, 1, 8, None) == _lib.H2O_ENOMEM
+    assert b"alloc" in _lib.lib.h2o_last_error(h)
+    # nothing stays allocated, the handle is still not prefilled
+    assert _lib.lib.h2o_step(h, dummy, dummy, dummy, dummy, 8, None) == _lib.H2O_ESTATE
+    assert _lib.lib.h2o_prefill(h, dummy, dummy, dummy, None, 1, 8, None) == _lib.H2O_ENOMEM
+    assert _lib.lib.h2o_destroy(h) == _lib.H2O_OK

@@ -57,6 +57,7 @@ def test_select_scatter_bytes():
 
 
 def test_reference_arm_prints_one_json_line():
+    # the reference arm on the default workload (28 layers, B=4): one oracle step per timed step
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                         "--steps", "1", "--warmup", "3"],
                        capture_output=True, text=True, timeout=600, cwd=ROOT)
@@ -68,3 +69,22 @@ def test_reference_arm_prints_one_json_line():
     assert d["metric"] == "H2O chunk-step query-tokens/s" and d["unit"] == "query-tokens/s"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["os_cpu_count"] == os.cpu_count()
+    # the same config object as the GPU arm prints, and the time it measured per step
+    b = _bench()
+    from h2o_kv_cache_b200.workload import CONFIGS
+    assert d["config"] == b.config_dict(CONFIGS[4], 1)
+    ex = d["extrapolation"]
+    assert abs(ex["ms_per_workload_step"] - d["ms_per_step"] * ex["caches_per_workload_step"]) < 1e-6 * ex["ms_per_workload_step"]
+    assert ex["caches_per_workload_step"] == 4 * 8 * 28
+
+
+def test_reference_arm_maps_no_product_library():
+    # the oracle arm loads the input generator from its file, not through the
+    # package (whose import loads libh2o.so)
+    code = ("import sys, runpy; sys.argv = ['bench.py', '--impl', 'reference', '--steps', '1', "
+            "'--warmup', '3', '--config', '0']; runpy.run_path('bench.py', run_name='__main__'); "
+            "maps = open('/proc/self/maps').read(); print('MAPPED' if 'libh2o' in maps else 'CLEAN')")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip().splitlines()[-1] == "CLEAN"

@@ -18,7 +18,7 @@ import torch
 
 from oracle import H2OHeadOracle, H2OOracle, select_evictions
 from tests.parity_util import (annotate_boundary, check_evictions, check_outputs, check_scores,
-                               to64)
+                               check_tie_state, to64)
 
 pytestmark = pytest.mark.gpu
 
@@ -94,6 +94,9 @@ def run_stream(h2o, cfg, heads=None, layer=0, T=None, oracle_chunks=None, kv_che
                                            check_scores(scores[b, h], st.score, st.pos >= 0, where))
             else:
                 summary["ties"] += 1
+                check_tie_state(slots[b, h], pos[b, h], pos_before[(b, h)], t0, where)
+                assert np.array_equal(d_evicted[b, h], pos_before[(b, h)][slots[b, h]]), \
+                    f"{where}: evicted positions differ"
                 # compare by position on the tokens both kept, then adopt the GPU state
                 gmap = {int(p): s for p, s in zip(pos[b, h], scores[b, h]) if p >= 0}
                 omap = {int(p): s for p, s in zip(st.pos, st.score) if p >= 0}
@@ -403,3 +406,34 @@ def test_standalone_select_reports_too_few_eligible(h2o):
     with pytest.raises(h2o.H2OError) as ei:
         h2o.select(scores, pos, t0=16, R=12, need=5)     # only pos 0..3 are eligible
     assert ei.value.status == -2
+
+
+@pytest.mark.parametrize("kind", ["alloc", "launch"])
+def test_host_fault_injection(h2o, monkeypatch, kind):
+    # faults made on the host (H2O_FAULT): an allocation that fails at prefill,
+    # a launch that fails at a step.  Each call reports its status and a message,
+    # the handle can be destroyed, and a fresh handle runs the stream at parity.
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    cfg = _cfg(0, dtype=torch.bfloat16, d=128)
+    Q, K, V = gen_batch(cfg, 0, device="cuda")
+    chunks = split_chunks(Q, K, V, cfg.bounds())
+    cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    if kind == "alloc":
+        monkeypatch.setenv("H2O_FAULT", "alloc")
+        with pytest.raises(h2o.H2OError) as ei:
+            cache.prefill(*chunks[0])
+        assert ei.value.status == -4 and "alloc" in str(ei.value)
+        monkeypatch.delenv("H2O_FAULT")
+        cache.prefill(*chunks[0])           # the failed prefill left nothing behind
+        assert cache.info()["t0"] == cfg.P
+    else:
+        cache.prefill(*chunks[0])
+        monkeypatch.setenv("H2O_FAULT", "launch")
+        with pytest.raises(h2o.H2OError) as ei:
+            cache.step(*chunks[1])
+        assert ei.value.status == -5 and "launch" in str(ei.value)
+        assert cache.info()["t0"] == cfg.P   # the failed step did not advance
+        monkeypatch.delenv("H2O_FAULT")
+    cache.close()
+    s = run_stream(h2o, cfg)
+    assert s["chunks"] == 5
