@@ -18,7 +18,7 @@ import torch
 from . import _lib
 from ._lib import (H2O_BF16, H2O_F32, H2O_OK, STATUS_NAMES, lib)
 
-__all__ = ["H2OCache", "H2OError", "select", "attend_noalloc", "lib"]
+__all__ = ["H2OCache", "H2OError", "select", "attend_noalloc", "step_layers", "lib"]
 
 _DTYPES = {torch.float32: H2O_F32, torch.bfloat16: H2O_BF16}
 
@@ -162,6 +162,34 @@ class H2OCache:
             self.close()
         except Exception:
             pass
+
+
+def step_layers(caches, qs, ks, vs, outs=None, stream=None):
+    """One chunk through several layers' caches (h2o_step_layers): the same result
+    as caches[l].step(qs[l], ks[l], vs[l], outs[l]) for every l, with one
+    attention launch and one tail launch for all layers when they share their
+    sizes.  Returns the list of outputs."""
+    n = len(caches)
+    if n < 1 or not (len(qs) == len(ks) == len(vs) == n):
+        raise ValueError("need one (q, k, v) per cache")
+    S = qs[0].shape[2]
+    if outs is None:
+        outs = [None] * n
+    outs = list(outs)
+    for l, c in enumerate(caches):
+        c._args(qs[l], ks[l], vs[l], S)
+        outs[l] = c._out(qs[l], outs[l])
+    dev = caches[0].device
+    if any(c.device != dev for c in caches):
+        raise ValueError("all caches must be on one device")
+    arr = lambda xs: (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])   # noqa: E731
+    hs = (ctypes.c_void_p * n)(*[c._h.value for c in caches])
+    with torch.cuda.device(dev):
+        _check(lib.h2o_step_layers(hs, n, arr(qs), arr(ks), arr(vs), arr(outs), S,
+                                   _stream_ptr(stream, dev)), caches[0]._h)
+    for c in caches:
+        c.last_S = S
+    return outs
 
 
 def select(scores, positions, t0: int, R: int, need: int, stream=None):

@@ -23,6 +23,8 @@ SIGNATURES = {
     "h2o_create": (_i32, [_i64, _i64, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp)]),
     "h2o_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _vp]),
     "h2o_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp]),
+    "h2o_step_layers": (_i32, [ctypes.POINTER(_vp), _i32, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                               ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i64, _vp]),
     "h2o_read_state": (_i32, [_vp, _vp, _vp, _vp, _vp]),
     "h2o_read_kv": (_i32, [_vp, _vp, _vp, _vp]),
     "h2o_read_delta": (_i32, [_vp, _vp, _vp, _vp]),

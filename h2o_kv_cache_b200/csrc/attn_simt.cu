@@ -12,7 +12,7 @@
 // One block = 64 query rows of one query head, one thread per row.  Two sweeps
 // over the visible keys: the first finds each row's log-sum-exp, the second
 // forms the exact probabilities p = exp(s - lse), accumulates out = p.V and
-// writes the block's column sums of p (a partial row of the summed weights).
+// adds the block's column sums of p to the (b, KV head)'s accumulator row.
 #include "h2o_internal.cuh"
 
 namespace h2o {
@@ -40,21 +40,20 @@ __global__ void __launch_bounds__(BR) attn_simt_kernel(AttnArgs a) {
   const int b = blockIdx.z;
   const int G = a.Hq / a.Hkv;
   const int h = g / G;
-  const int gl = g - h * G;
   const int64_t S = a.S, M = a.M, nv = a.n_valid;
   const int64_t i0 = (int64_t)rt * BR;
   const int64_t i = i0 + tid;
   const bool row_ok = i < S;
-  const int n_rt = (int)((S + BR - 1) / BR);
 
   const T* qb = static_cast<const T*>(a.q) + ((int64_t)b * a.Hq + g) * S * D;
   const T* kb = static_cast<const T*>(a.k) + ((int64_t)b * a.Hkv + h) * S * D;
   const T* vb = static_cast<const T*>(a.v) + ((int64_t)b * a.Hkv + h) * S * D;
   const T* kcb = static_cast<const T*>(a.kc) + ((int64_t)b * a.Hkv + h) * M * D;
   const T* vcb = static_cast<const T*>(a.vc) + ((int64_t)b * a.Hkv + h) * M * D;
-  float* part = a.partials + (((int64_t)b * a.Hkv + h) * (G * n_rt) + (gl * n_rt + rt)) * a.part_stride;
+  unsigned long long* acc_row = a.colacc + ((int64_t)b * a.Hkv + h) * a.acc_stride;
+  const float fx_scale = __int_as_float((127 + a.fx_shift) << 23);   // 2^fx_shift
 
-  // the cache and the partial rows may still be in use by the previous kernel
+  // the cache and the accumulator row may still be in use by the previous kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   for (int e = tid; e < BR * D; e += BR) {
@@ -128,7 +127,7 @@ __global__ void __launch_bounds__(BR) attn_simt_kernel(AttnArgs a) {
         if (kk < key_lim) {
           float cs = 0.f;
           for (int r = 0; r < BR; ++r) cs += Ps[r * (BK + 1) + tid];
-          part[is_cache ? kk : M + kk] = cs;
+          colsum_add(acc_row + (is_cache ? kk : M + kk), cs, fx_scale);
         }
       }
     }

@@ -8,8 +8,11 @@
 // A unit of work is the 128 rows of two query heads (as in attn_umma.cu) and
 // its keys, counted in 256-key pairs.  Units differ in size (the causal part
 // of the chunk), and 128 or 256 of them on 148 SMs leave SMs idle.  Here the
-// pairs of all units form one sequence that is cut into n_cta equal runs; CTA
-// i takes run i, i.e. the end of one unit, whole units, and the start of
+// units are taken in rounds of whole KV heads, as many heads a round as keep
+// their K and V within half of L2 (every CTA works on the same few heads at a
+// time, so the second sweep's K and V come from L2); the pairs of a round's
+// units form one sequence that is cut into n_cta equal runs, and CTA i takes
+// run i of every round: the end of one unit, whole units, and the start of
 // another.  Each part of a unit in one CTA is a "piece".
 //   kernel A (sweep 1): per piece, S = Q K^T and each row's running (max, sum)
 //            over the piece's keys -> global workspace [unit][piece][row];
@@ -24,7 +27,7 @@
 // four softmax warpgroups: in kernel A each takes a quarter of every 256-key
 // tile's keys for both heads (the four (max, sum) are merged per piece); in
 // kernel B each takes 64 query columns of S^T, which is two 128-column
-// buffers, one per head, and writes its own partial row of column sums.
+// buffers, one per head, and adds its column sums to the accumulator row.
 // Every mbarrier wait is bounded.
 #include <cstdio>
 #include <vector>
@@ -40,7 +43,6 @@ using namespace attn;
 constexpr int kWg = 4;                           // softmax warpgroups (both kernels)
 constexpr int kSoft = 128 * kWg;                 // softmax threads
 constexpr int kThreads = 64 + kSoft;             // + TMA producer warp + MMA warp
-static_assert(kWg == kStreamRows, "one partial row per softmax warpgroup");
 constexpr int kMaxPieces = 8;                    // per CTA (the host checks)
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr uint32_t kTmemCols = 512;
@@ -85,18 +87,18 @@ constexpr uint32_t kB_SmemBytes = kB_OffBar + B_NUM * 8 + kMiscBytes + 1024;
 static_assert(kA_SmemBytes <= 232448 && kB_SmemBytes <= 232448, "shared memory budget");
 
 struct SParams {
-  float* partials;      // column sums, [BHkv][n_pg * n_rt][stride]
+  unsigned long long* colacc;   // fixed-point summed weights, [BHkv][acc_stride]
   int* err;
   void* out;            // [B, Hq, S, D] bf16, or null
   float2* ws_ml;        // [units][maxp][2 * BM]: a piece's rows' (max, sum), base 2
   float* ws_o;          // [units][maxp][2 * BM][D]: a piece's partial O (split units)
   int* count;           // [units]: pieces of the unit done with sweep 2
   int B, Hq, Hkv, G, n_pg, n_rt, maxp;
-  int n_grp;            // partial rows per (b, KV head, row tile): kStreamRows per head pair
   int inject_timeout;   // test hook: one wait of kernel B runs out
-  int64_t S, M, n_valid, stride;
-  int64_t total_pairs;  // over all units
+  int64_t S, M, n_valid, acc_stride;
+  int heads_per_round;  // (b, KV head) caches per round
   float scale_log2;
+  float fx_scale;       // 2^fx_shift of the accumulator
 };
 
 // ---- units: u = (bh * n_pg + pg) * n_rt + rt
@@ -125,33 +127,39 @@ __device__ __forceinline__ UnitGeo unit_geo(const SParams& p, int u) {
 __device__ __forceinline__ int unit_pairs(const SParams& p, int u) {
   return (unit_geo(p, u).n_all + 1) >> 1;
 }
-// CTA whose run holds global pair g: runs start at floor(i * P / n_cta)
-__device__ __forceinline__ int cta_of(int64_t g, int64_t P, int n_cta) {
+// CTA whose run holds pair g of a round of P pairs: runs start at floor(i * P / n_cta)
+__host__ __device__ __forceinline__ int cta_of(int64_t g, int64_t P, int n_cta) {
   return (int)(((g + 1) * n_cta + P - 1) / P) - 1;
 }
 
-// Thread 0: this CTA's pieces into shared memory; returns their number.
+// Thread 0: this CTA's pieces into shared memory, round after round; returns
+// their number (-1 if more than kMaxPieces).
 __device__ int build_pieces(const SParams& p, Piece* pc) {
   const int n_cta = gridDim.x;
-  const int64_t P = p.total_pairs;
-  const int64_t lo = (int64_t)blockIdx.x * P / n_cta, hi = (int64_t)(blockIdx.x + 1) * P / n_cta;
-  const int units = p.B * p.Hkv * p.n_pg * p.n_rt;
+  const int BH = p.B * p.Hkv, per_head = p.n_pg * p.n_rt;
   int n = 0;
-  int64_t g0 = 0;   // first global pair of unit u
-  for (int u = 0; u < units && g0 < hi; ++u) {
-    const int q = unit_pairs(p, u);
-    const int64_t g1 = g0 + q;
-    if (g1 > lo) {
-      if (n == kMaxPieces) return -1;
-      Piece& x = pc[n++];
-      x.u = u;
-      x.a = (int)((lo > g0 ? lo : g0) - g0);
-      x.c = (int)((hi < g1 ? hi : g1) - g0);
-      const int first = cta_of(g0, P, n_cta), last = cta_of(g1 - 1, P, n_cta);
-      x.k = (int)blockIdx.x - first;
-      x.np = last - first + 1;
+  for (int h0 = 0; h0 < BH; h0 += p.heads_per_round) {
+    const int u_lo = h0 * per_head;
+    const int u_hi = (h0 + p.heads_per_round < BH ? h0 + p.heads_per_round : BH) * per_head;
+    int64_t P = 0;
+    for (int u = u_lo; u < u_hi; ++u) P += unit_pairs(p, u);
+    const int64_t lo = (int64_t)blockIdx.x * P / n_cta, hi = (int64_t)(blockIdx.x + 1) * P / n_cta;
+    int64_t g0 = 0;   // first pair of unit u within the round
+    for (int u = u_lo; u < u_hi && g0 < hi; ++u) {
+      const int q = unit_pairs(p, u);
+      const int64_t g1 = g0 + q;
+      if (g1 > lo) {
+        if (n == kMaxPieces) return -1;
+        Piece& x = pc[n++];
+        x.u = u;
+        x.a = (int)((lo > g0 ? lo : g0) - g0);
+        x.c = (int)((hi < g1 ? hi : g1) - g0);
+        const int first = cta_of(g0, P, n_cta), last = cta_of(g1 - 1, P, n_cta);
+        x.k = (int)blockIdx.x - first;
+        x.np = last - first + 1;
+      }
+      g0 = g1;
     }
-    g0 = g1;
   }
   return n;
 }
@@ -542,7 +550,7 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // =========================================================== softmax / epilogue
     // Four warpgroups: warpgroup wg takes the 64 query columns [64 wg, 64 wg + 64)
     // of S^T, i.e. queries [64 hq, 64 hq + 64) of head w (w = wg / 2, hq = wg % 2),
-    // and writes its own partial row of column sums.
+    // and adds its column sums of them to the accumulator row.
     const int wg = (warp - 2) >> 2;
     const int w = wg >> 1, hq = wg & 1;
     const int quarter = warp & 3;
@@ -590,7 +598,7 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         nlse[wg * BM + r] = (row_head_ok && row_i < S && lsum > 0.f) ? -(mx + lg2(lsum)) : -INFINITY;
       }
       named_bar_sync(1, kSoft);
-      float* part = p.partials + ((int64_t)g.bh * (p.n_grp * p.n_rt) + ((g.pg * kStreamRows + wg) * p.n_rt + g.rt)) * p.stride;
+      unsigned long long* acc = p.colacc + (int64_t)g.bh * p.acc_stride;
       for (int j = 0; ok && j < n; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ST_FULL + w), (uint32_t)st & 1u, abort_flag, p.err,
                                                kWaitLimitNs, kErrTimeout));
@@ -626,7 +634,7 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         fence_async_smem();
         mbar_arrive(bar(B_P_FULL));
         // without a head B every p of warpgroups 2 and 3 is 0
-        if (key_ok) part[cache ? key : M + key] = head_ok ? cs_total(cs4) : 0.f;
+        if (key_ok && head_ok) colsum_add(acc + (cache ? key : M + key), cs_total(cs4), p.fx_scale);
         ++st;
       }
       // ----- the piece's O^T (lane = d, columns = the warpgroup's 64 queries of head w)
@@ -723,11 +731,29 @@ attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 }  // namespace
 
+// (b, KV head) caches per round: as many as keep their K and V rows (those
+// the step reads) within half of L2, at least one; rounds of equal size.
+int heads_per_round(const AttnArgs& a) {
+  const int BH = a.B * a.Hkv;
+  int l2 = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return BH;
+  }
+  const double kv = (double)(a.n_valid + a.S) * D * 2.0 * 2.0;   // bf16 K and V of one cache
+  int h = (int)(0.5 * l2 / kv);
+  if (h < 1) h = 1;
+  if (h >= BH) return BH;
+  const int rounds = (BH + h - 1) / h;
+  return (BH + rounds - 1) / rounds;
+}
+
 bool attn_stream_plan(const AttnArgs& a, int n_sm, StreamPlan* pl) {
   if (!attn_umma_supported(kBF16, a.d) || n_sm < 1 || a.S < 1) return false;
   const int G = a.Hq / a.Hkv, n_pg = (G + 1) / 2;
   const int n_rt = (int)((a.S + BM - 1) / BM);
-  const int64_t units = (int64_t)a.B * a.Hkv * n_pg * n_rt;
+  const int BH = a.B * a.Hkv, per_head = n_pg * n_rt;
+  const int64_t units = (int64_t)BH * per_head;
   if (units < 1 || units > (1 << 24)) return false;
   const int nct = (int)((a.n_valid + BN - 1) / BN);
   std::vector<int> q((size_t)units);
@@ -739,22 +765,35 @@ bool attn_stream_plan(const AttnArgs& a, int n_sm, StreamPlan* pl) {
     q[(size_t)u] = (n_all + 1) >> 1;
     P += q[(size_t)u];
   }
-  const int n_cta = (int)(P < n_sm ? P : n_sm);
-  auto cta_of_h = [&](int64_t g) { return (int)(((g + 1) * n_cta + P - 1) / P) - 1; };
+  const int hpr = heads_per_round(a);
+  // every round is cut into n_cta runs; with fewer pairs than SMs in a round,
+  // n_cta is that round's pair count at most
+  int n_cta = n_sm;
+  for (int h0 = 0; h0 < BH; h0 += hpr) {
+    int64_t Pr = 0;
+    for (int u = h0 * per_head; u < (h0 + hpr < BH ? h0 + hpr : BH) * per_head; ++u) Pr += q[(size_t)u];
+    if (Pr < n_cta) n_cta = (int)Pr;
+  }
   std::vector<int> per_cta((size_t)n_cta, 0);
   int maxp = 1;
-  int64_t g0 = 0;
-  for (int64_t u = 0; u < units; ++u) {
-    const int first = cta_of_h(g0), last = cta_of_h(g0 + q[(size_t)u] - 1);
-    if (last - first + 1 > maxp) maxp = last - first + 1;
-    for (int i = first; i <= last; ++i)
-      if (++per_cta[(size_t)i] > kMaxPieces) return false;
-    g0 += q[(size_t)u];
+  for (int h0 = 0; h0 < BH; h0 += hpr) {
+    const int u_lo = h0 * per_head, u_hi = (h0 + hpr < BH ? h0 + hpr : BH) * per_head;
+    int64_t Pr = 0;
+    for (int u = u_lo; u < u_hi; ++u) Pr += q[(size_t)u];
+    int64_t g0 = 0;
+    for (int u = u_lo; u < u_hi; ++u) {
+      const int first = cta_of(g0, Pr, n_cta), last = cta_of(g0 + q[(size_t)u] - 1, Pr, n_cta);
+      if (last - first + 1 > maxp) maxp = last - first + 1;
+      for (int i = first; i <= last; ++i)
+        if (++per_cta[(size_t)i] > kMaxPieces) return false;
+      g0 += q[(size_t)u];
+    }
   }
   pl->n_cta = n_cta;
   pl->maxp = maxp;
   pl->units = (int)units;
   pl->total_pairs = P;
+  pl->heads_per_round = hpr;
   pl->ml_bytes = (size_t)units * maxp * 2 * BM * sizeof(float2);
   pl->o_bytes = maxp > 1 ? (size_t)units * maxp * 2 * BM * D * sizeof(float) : 0;
   pl->count_bytes = (size_t)units * sizeof(int);
@@ -776,7 +815,7 @@ cudaError_t launch_attn_stream(const AttnArgs& a, const StreamPlan& pl, void* ws
   if ((e = make_map(&mkc, has_cache ? a.kc : a.k, has_cache ? a.M : a.S, BHkv)) != cudaSuccess) return e;
   if ((e = make_map(&mvc, has_cache ? a.vc : a.v, has_cache ? a.M : a.S, BHkv)) != cudaSuccess) return e;
   SParams p;
-  p.partials = a.partials;
+  p.colacc = a.colacc;
   p.err = a.err;
   p.out = a.out;
   p.ws_ml = static_cast<float2*>(ws_ml);
@@ -789,13 +828,13 @@ cudaError_t launch_attn_stream(const AttnArgs& a, const StreamPlan& pl, void* ws
   p.n_pg = (p.G + 1) / 2;
   p.n_rt = (int)((a.S + BM - 1) / BM);
   p.maxp = pl.maxp;
-  p.n_grp = stream_partial_groups(p.G);
   p.inject_timeout = a.inject_timeout;
   p.S = a.S;
   p.M = a.M;
   p.n_valid = a.n_valid;
-  p.stride = a.part_stride;
-  p.total_pairs = pl.total_pairs;
+  p.acc_stride = a.acc_stride;
+  p.fx_scale = fx_scale_of(a.fx_shift);
+  p.heads_per_round = pl.heads_per_round;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   if ((e = cudaFuncSetAttribute(lse_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kA_SmemBytes)) != cudaSuccess)

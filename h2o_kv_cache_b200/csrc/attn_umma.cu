@@ -16,7 +16,8 @@
 //            p = exp(s - lse) for its head's 128 queries, sums them (its column
 //            sum, no cross-thread reduction) and writes them to shared memory
 //            as P^T; then O^T += V^T P^T (M = 128 = d, N = 256 queries), both
-//            operands MN-major.
+//            operands MN-major.  Each key's column sum of each head is added
+//            to the (b, KV head)'s fixed-point accumulator row.
 // Split keys: a unit of work (two heads' 128 rows) may be shared by a cluster
 // of kc CTAs, each taking a contiguous run of its 256-key pairs.  After sweep 1
 // every CTA publishes its rows' (max, sum) in shared memory, and each CTA
@@ -28,8 +29,7 @@
 // grids that would leave a partial last wave use kc > 1.
 // Exact probabilities mean O needs no rescaling.  Every MMA has N = 256: with
 // both operands in shared memory that is what keeps the tensor core near its
-// peak (N = 128 runs at about 70% of it).  Each (head, key) column sum of the
-// CTA goes to one partial row that a fixed-order reduction adds up.
+// peak (N = 128 runs at about 70% of it).
 //
 // Warp roles (320 threads): warp 0 issues TMA loads (one thread), warp 1
 // allocates TMEM and issues the MMAs (one thread), warps 2-5 / 6-9 are two
@@ -44,6 +44,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "attn_common.cuh"
@@ -68,8 +69,7 @@ constexpr uint32_t kOffLse = kOffR + kRBytes;           // negated base-2 lse, [
 constexpr uint32_t kOffBar = kOffLse + 2 * BM * 4;
 constexpr int kNumBars = 26;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kOffCs = kOffMisc + 16;             // head B's column sums of a tile, [128]
-constexpr uint32_t kSmemUsed = kOffCs + BN * 4;
+constexpr uint32_t kSmemUsed = kOffMisc + 16;
 // cluster exchange of sweep-1 (max, sum) pairs, [2][128] float2: the part of
 // R that neither the sweep-1 slots nor the sweep-2 ring use, and that P^T
 // first overwrites only after every CTA of the cluster has read it
@@ -90,26 +90,38 @@ constexpr uint32_t kDescHi = desc_hi_sw128(1024);   // 8 rows of 128 bytes betwe
 enum { B_Q = 0, B_R1_FULL = 1, B_R1_EMPTY = 3, B_R2_FULL = 5, B_R2_EMPTY = B_R2_FULL + NS2,
        B_S_FULL = B_R2_EMPTY + NS2, B_S_EMPTY = B_S_FULL + 2, B_ST_FULL = B_S_EMPTY + 2,
        B_ST_EMPTY = B_ST_FULL + 1, B_P_FULL = B_ST_EMPTY + 1, B_P_EMPTY = B_P_FULL + 1,
-       B_O_FULL = B_P_EMPTY + 1, B_DRAIN = B_O_FULL + 1, B_CS_FULL = B_DRAIN + 1,
-       B_CS_EMPTY = B_CS_FULL + 1, B_X_READY = B_CS_EMPTY + 1, B_X_READ = B_X_READY + 1,
+       B_O_FULL = B_P_EMPTY + 1, B_DRAIN = B_O_FULL + 1, B_X_READY = B_DRAIN + 1,
+       B_X_READ = B_X_READY + 1,
        B_NEVER = B_X_READ + 1 };   // test hook: nothing ever arrives on it
 static_assert(B_NEVER < kNumBars, "barrier count");
 
 struct Params {
-  float* partials;
+  unsigned long long* colacc;      // [B * Hkv][acc_stride] fixed-point summed weights
   int* err;
   void* out;
   int B, Hq, Hkv, G, n_pg, n_rt;
+  int units;                       // units of work per layer
   int kc;                          // CTAs (a cluster) per unit of work
   int inject_timeout;              // test hook: make one wait run out
-  int64_t S, M, n_valid, stride;   // stride: floats between partial rows
+  int64_t S, M, n_valid, acc_stride;
   float scale_log2;   // (1/sqrt(d)) * log2(e)
+  float fx_scale;     // 2^fx_shift of the accumulator
 };
 
+// A group of L layers that share every size: per layer its five tensor maps
+// (q, k, v, cache k, cache v) and its parameters.  One grid covers all the
+// layers' units, layer after layer, so a partial last wave is paid once per
+// group instead of once per layer.
+constexpr int kMaxGroup = 32;
+template <int L>
+struct Group {
+  CUtensorMap maps[L][5];
+  Params p[L];
+};
+
+template <int L>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
-                 const __grid_constant__ CUtensorMap tm_vc, const Params p) {
+attn_umma_kernel(const __grid_constant__ Group<L> grp) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -121,10 +133,24 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work unit: (b, h) major, then row tiles from the last (heaviest), then head pairs
-  const int kc = p.kc;
+  // ---- work unit: layer, then (b, h), then row tiles from the last (heaviest), then head pairs
+  const int kc = grp.p[0].kc;
   const int rank = (int)(blockIdx.x % (unsigned)kc);        // rank in the cluster
-  const int unit = (int)(blockIdx.x / (unsigned)kc);
+  const int unit_g = (int)(blockIdx.x / (unsigned)kc);
+  const int layer = L == 1 ? 0 : unit_g / grp.p[0].units;
+  const int unit = unit_g - layer * grp.p[0].units;
+  // sizes are the same in every layer of the group (read from layer 0's
+  // parameters, which the compiler addresses directly); per layer only the
+  // output, the accumulator row and the error word differ
+  const Params& p = grp.p[0];
+  int* const err = grp.p[layer].err;
+  void* const out = grp.p[layer].out;
+  unsigned long long* const colacc = grp.p[layer].colacc;
+  const CUtensorMap* const tm_q = &grp.maps[layer][0];
+  const CUtensorMap* const tm_k = &grp.maps[layer][1];
+  const CUtensorMap* const tm_v = &grp.maps[layer][2];
+  const CUtensorMap* const tm_kc = &grp.maps[layer][3];
+  const CUtensorMap* const tm_vc = &grp.maps[layer][4];
   const int per_bh = p.n_pg * p.n_rt;
   const int bh = unit / per_bh;
   const int k_in = unit - bh * per_bh;
@@ -152,7 +178,6 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       uint32_t cnt = 1;
       if (i == B_S_EMPTY || i == B_S_EMPTY + 1) cnt = 256;   // both warpgroups
       if (i == B_ST_EMPTY || i == B_P_FULL) cnt = 256;        // both warpgroups
-      if (i == B_CS_FULL || i == B_CS_EMPTY) cnt = 128;       // one warpgroup
       if (i == B_X_READY || i == B_X_READ) cnt = (uint32_t)kc;  // one arrival per CTA
       mbar_init(bar(i), cnt);
     }
@@ -168,20 +193,20 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (kc > 1) cluster_sync_all();   // every CTA's barriers exist before remote arrivals
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // the cache and the partial rows may still be in use by the previous kernel
+  // the cache and the accumulator row may still be in use by the previous kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // local tile t (128 keys), i.e. the unit's tile t_lo + t: tensor map and row offset
   auto tile_src = [&](int t, bool v, const CUtensorMap*& m, int& y) {
     const int tg = t_lo + t;
     if (tg < nct) {
-      m = v ? &tm_vc : &tm_kc;
+      m = v ? tm_vc : tm_kc;
       y = tg * BN;
     } else if (tg < t_hi) {
-      m = v ? &tm_v : &tm_k;
+      m = v ? tm_v : tm_k;
       y = (tg - nct) * BN;
     } else {  // past the last tile: a box beyond the chunk's rows reads zeros
-      m = v ? &tm_v : &tm_k;
+      m = v ? tm_v : tm_k;
       y = (int)p.S;
     }
   };
@@ -189,24 +214,24 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (warp == 0) {
     // =========================================================== TMA producer
     if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      prefetch_tmap(&tm_kc);
-      prefetch_tmap(&tm_vc);
+      prefetch_tmap(tm_q);
+      prefetch_tmap(tm_k);
+      prefetch_tmap(tm_v);
+      prefetch_tmap(tm_kc);
+      prefetch_tmap(tm_vc);
       // Q: rows of head A then head B, each split into two 64-column atoms
       const int zq = b * p.Hq + h * p.G + gl_a;
       mbar_arrive_expect_tx(bar(B_Q), 2 * kTile);
       for (int hw = 0; hw < 2; ++hw)
         for (int at = 0; at < 2; ++at)
-          tma_load_3d(base + kOffQ + at * 2 * kAtom + hw * kAtom, &tm_q, bar(B_Q), at * 64, (int)i0,
+          tma_load_3d(base + kOffQ + at * 2 * kAtom + hw * kAtom, tm_q, bar(B_Q), at * 64, (int)i0,
                       zq + hw);
       bool ok = true;
       int issued1 = 0;                               // sweep-1 tiles whose loads were issued
       // sweep 1: 256-key K tiles into two 64 KB slots
       for (int u = 0; ok && u < n1; ++u) {
         const int s = u & 1;
-        ok = mbar_wait(bar(B_R1_EMPTY + s), ((uint32_t)(u >> 1) & 1u) ^ 1u, abort_flag, p.err,
+        ok = mbar_wait(bar(B_R1_EMPTY + s), ((uint32_t)(u >> 1) & 1u) ^ 1u, abort_flag, err,
                        kWaitLimitNs, kErrTimeout);
         if (!ok) break;
         const uint32_t dst = base + kOffR + (uint32_t)s * kSlot1;
@@ -224,13 +249,13 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int s = 0; ok && s < 2; ++s) {
         const int fills = (n1 - s + 1) >> 1;
         if (fills > 0)
-          ok = mbar_wait(bar(B_R1_EMPTY + s), (uint32_t)(fills - 1) & 1u, abort_flag, p.err,
+          ok = mbar_wait(bar(B_R1_EMPTY + s), (uint32_t)(fills - 1) & 1u, abort_flag, err,
                          kWaitLimitNs, kErrTimeout);
       }
       int issued = 0;
       for (int pos = 0; ok && pos < 2 * n; ++pos) {
         const int slot = pos % NS2;
-        ok = mbar_wait(bar(B_R2_EMPTY + slot), ((uint32_t)(pos / NS2) & 1u) ^ 1u, abort_flag, p.err,
+        ok = mbar_wait(bar(B_R2_EMPTY + slot), ((uint32_t)(pos / NS2) & 1u) ^ 1u, abort_flag, err,
                        kWaitLimitNs, kErrTimeout);
         if (!ok) break;
         bool is_v;
@@ -249,11 +274,11 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         issued = pos + 1;
       }
       // drain, also after an abort: every load issued has landed before the CTA may exit
-      mbar_drain(bar(B_Q), 0, p.err, kWaitLimitNs, kErrTimeout);
+      mbar_drain(bar(B_Q), 0, err, kWaitLimitNs, kErrTimeout);
       for (int u = issued1 - 2 < 0 ? 0 : issued1 - 2; u < issued1; ++u)
-        mbar_drain(bar(B_R1_FULL + (u & 1)), (uint32_t)(u >> 1) & 1u, p.err, kWaitLimitNs, kErrTimeout);
+        mbar_drain(bar(B_R1_FULL + (u & 1)), (uint32_t)(u >> 1) & 1u, err, kWaitLimitNs, kErrTimeout);
       for (int pos = issued - NS2 < 0 ? 0 : issued - NS2; pos < issued; ++pos)
-        mbar_drain(bar(B_R2_FULL + pos % NS2), (uint32_t)(pos / NS2) & 1u, p.err, kWaitLimitNs,
+        mbar_drain(bar(B_R2_FULL + pos % NS2), (uint32_t)(pos / NS2) & 1u, err, kWaitLimitNs,
                    kErrTimeout);
     }
   } else if (warp == 1) {
@@ -263,15 +288,15 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const uint32_t idesc_mn = idesc_bf16(128, 256, 1, 1);   // both operands MN-major
       const uint32_t q_addr = base + kOffQ;
       const uint32_t p_addr = base + kOffP;
-      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, p.err, kWaitLimitNs, kErrTimeout);
+      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, err, kWaitLimitNs, kErrTimeout);
       // ---- sweep 1
       for (int u = 0; ok && u < n1; ++u) {
         const int s = u & 1;
-        ok = mbar_wait(bar(B_R1_FULL + s), (uint32_t)(u >> 1) & 1u, abort_flag, p.err, kWaitLimitNs,
+        ok = mbar_wait(bar(B_R1_FULL + s), (uint32_t)(u >> 1) & 1u, abort_flag, err, kWaitLimitNs,
                        kErrTimeout);
         const uint32_t k_addr = base + kOffR + (uint32_t)s * kSlot1;
         for (int w = 0; ok && w < 2; ++w) {
-          ok = mbar_wait(bar(B_S_EMPTY + w), ((uint32_t)u & 1u) ^ 1u, abort_flag, p.err, kWaitLimitNs,
+          ok = mbar_wait(bar(B_S_EMPTY + w), ((uint32_t)u & 1u) ^ 1u, abort_flag, err, kWaitLimitNs,
                          kErrTimeout);
           if (!ok) break;
           tc_fence_after();
@@ -288,11 +313,11 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       auto issue_st = [&](int j) -> bool {
         // TMEM columns 0-255: head A's last sweep-1 S, then S^T(j - 1), must have been read
         bool w_ok = (j == 0)
-            ? mbar_wait(bar(B_S_EMPTY + 0), ((uint32_t)n1 & 1u) ^ 1u, abort_flag, p.err, kWaitLimitNs, kErrTimeout)
-            : mbar_wait(bar(B_ST_EMPTY), (uint32_t)(j - 1) & 1u, abort_flag, p.err, kWaitLimitNs, kErrTimeout);
+            ? mbar_wait(bar(B_S_EMPTY + 0), ((uint32_t)n1 & 1u) ^ 1u, abort_flag, err, kWaitLimitNs, kErrTimeout)
+            : mbar_wait(bar(B_ST_EMPTY), (uint32_t)(j - 1) & 1u, abort_flag, err, kWaitLimitNs, kErrTimeout);
         const int pos = k_pos(j), slot = pos % NS2;
         if (w_ok)
-          w_ok = mbar_wait(bar(B_R2_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, p.err,
+          w_ok = mbar_wait(bar(B_R2_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, err,
                            kWaitLimitNs, kErrTimeout);
         if (!w_ok) return false;
         tc_fence_after();
@@ -306,14 +331,14 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         return true;
       };
       auto issue_ot = [&](int j) -> bool {
-        bool w_ok = mbar_wait(bar(B_P_FULL), (uint32_t)j & 1u, abort_flag, p.err, kWaitLimitNs, kErrTimeout);
+        bool w_ok = mbar_wait(bar(B_P_FULL), (uint32_t)j & 1u, abort_flag, err, kWaitLimitNs, kErrTimeout);
         // TMEM columns 256-511: head B's last sweep-1 S must have been read
         if (w_ok && j == 0)
-          w_ok = mbar_wait(bar(B_S_EMPTY + 1), ((uint32_t)n1 & 1u) ^ 1u, abort_flag, p.err,
+          w_ok = mbar_wait(bar(B_S_EMPTY + 1), ((uint32_t)n1 & 1u) ^ 1u, abort_flag, err,
                            kWaitLimitNs, kErrTimeout);
         const int pos = v_pos(n, j), slot = pos % NS2;
         if (w_ok)
-          w_ok = mbar_wait(bar(B_R2_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, p.err,
+          w_ok = mbar_wait(bar(B_R2_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, err,
                            kWaitLimitNs, kErrTimeout);
         if (!w_ok) return false;
         tc_fence_after();
@@ -334,7 +359,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       umma_commit(bar(B_O_FULL));
       // every MMA issued has completed before TMEM is released, also after an abort
       umma_commit(bar(B_DRAIN));
-      mbar_drain(bar(B_DRAIN), 0, p.err, kWaitLimitNs, kErrTimeout);
+      mbar_drain(bar(B_DRAIN), 0, err, kWaitLimitNs, kErrTimeout);
     }
   } else {
     // =========================================================== softmax / epilogue
@@ -349,7 +374,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (p.inject_timeout && w == 0) {
       // test hook: a bounded wait on a barrier nothing completes runs out (1 ms);
       // every role then leaves through its abort path and the step reports it
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_NEVER), 0, abort_flag, p.err, 1000000ull, kErrTimeout));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_NEVER), 0, abort_flag, err, 1000000ull, kErrTimeout));
     }
 
     // ----- sweep 1: both warpgroups read each head's S tile, warpgroup w
@@ -374,7 +399,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int u = 0; ok && u < n1; ++u) {
 #pragma unroll
       for (int hw = 0; hw < 2; ++hw) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + hw), (uint32_t)u & 1u, abort_flag, p.err,
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + hw), (uint32_t)u & 1u, abort_flag, err,
                                                kWaitLimitNs, kErrTimeout));
         if (!ok) break;
         tc_fence_after();
@@ -421,7 +446,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         asm volatile("fence.acq_rel.cluster;" ::: "memory");
         for (int q = 0; q < kc; ++q) mbar_arrive_remote(cluster_map(bar(B_X_READY), (uint32_t)q));
       }
-      ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_X_READY), 0, abort_flag, p.err, kWaitLimitNs,
+      ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_X_READY), 0, abort_flag, err, kWaitLimitNs,
                                                    kErrTimeout));
       float mq[kMaxSplit], lq[kMaxSplit];
       float mx = -INFINITY;
@@ -448,31 +473,18 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     named_bar_sync(1 + w, 128);
 
-    // ----- sweep 2: thread = key (lane r of S^T), the 128 query columns of head w
-    // One partial row per (head pair, row tile): warpgroup 1 hands head B's
-    // column sum of each key to warpgroup 0 through cs_b, which stores the
-    // sum of the two (an exact two-term add) one tile later.
-    float* part = p.partials + ((int64_t)bh * (p.n_pg * p.n_rt) + (pg * p.n_rt + rt)) * p.stride;
-    float* cs_b = reinterpret_cast<float*>(sbase + kOffCs);
-    float prev_cs = 0.f;
-    int64_t prev_col = -1;
+    // ----- sweep 2: thread = key (lane r of S^T), the 128 query columns of head w;
+    // each warpgroup adds its head's column sum of the key to the accumulator row
+    unsigned long long* acc = colacc + (int64_t)bh * p.acc_stride;
     const uint32_t p_row = base + kOffP + (uint32_t)(2 * w) * kAtom + (uint32_t)(r >> 3) * 1024u +
                            (uint32_t)(r & 7) * 128u;
     const float* nl_w = nlse + w * BM;
     const uint32_t st_tmem = lane_base + (uint32_t)w * 128u;
     for (int j = 0; ok && j < n; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ST_FULL), (uint32_t)j & 1u, abort_flag, p.err,
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ST_FULL), (uint32_t)j & 1u, abort_flag, err,
                                              kWaitLimitNs, kErrTimeout));
       if (!ok) break;
       tc_fence_after();
-      if (w == 0 && j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_FULL), (uint32_t)(j - 1) & 1u, abort_flag,
-                                               p.err, kWaitLimitNs, kErrTimeout));
-        if (!ok) break;
-        const float other = cs_b[r];
-        mbar_arrive(bar(B_CS_EMPTY));
-        if (prev_col >= 0) part[prev_col] = prev_cs + other;
-      }
       const int jg = t_lo + j;
       const bool cache = jg < nct;
       const int64_t key = cache ? (int64_t)jg * BN + r : (int64_t)(jg - nct) * BN + r;
@@ -504,39 +516,24 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         else key_half<false>(v, nl_w + 64, c, key_ok, qmin - 64, cs4, pk2);
       }
       if (kc > 1 && j == 0) {   // the cluster is done with the exchange area
-        ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_X_READ), 0, abort_flag, p.err,
+        ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_X_READ), 0, abort_flag, err,
                                                      kWaitLimitNs, kErrTimeout));
         if (!ok) break;
       }
       // this warpgroup's P^T half of the previous tile has been read by its O^T MMA
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
-                                             p.err, kWaitLimitNs, kErrTimeout));
+                                             err, kWaitLimitNs, kErrTimeout));
       if (!ok) break;
       store_p_half(p_row, r, pk);
       store_p_half(p_row + kAtom, r, pk2);
       fence_async_smem();
       mbar_arrive(bar(B_P_FULL));
-      const float cs = cs_total(cs4);
-      if (w == 0) {
-        prev_cs = cs;
-        prev_col = key_ok ? (cache ? key : M + key) : -1;
-      } else {
-        // without a head B every probability of this warpgroup is 0
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
-                                               p.err, kWaitLimitNs, kErrTimeout));
-        if (!ok) break;
-        cs_b[r] = head_ok ? cs : 0.f;
-        mbar_arrive(bar(B_CS_FULL));
-      }
-    }
-    if (w == 0 && ok && n > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CS_FULL), (uint32_t)(n - 1) & 1u, abort_flag,
-                                             p.err, kWaitLimitNs, kErrTimeout));
-      if (ok && prev_col >= 0) part[prev_col] = prev_cs + cs_b[r];
+      // without a head B every probability of warpgroup 1 is 0
+      if (key_ok && head_ok) colsum_add(acc + (cache ? key : M + key), cs_total(cs4), p.fx_scale);
     }
 
     // ----- epilogue: O^T (lane = d, columns = queries) -> out rows via shared memory
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), 0, abort_flag, p.err,
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), 0, abort_flag, err,
                                                    kWaitLimitNs, kErrTimeout));
     if (kc == 1) {
       // every MMA has completed: R is free; head w's [128 queries x 128 d] goes to R + w * 32 KB.
@@ -556,9 +553,9 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       named_bar_sync(1 + w, 128);
       const int64_t qi = i0 + r;                       // thread r copies query row r
-      if (ok && p.out != nullptr && head_ok && qi < S) {
+      if (ok && out != nullptr && head_ok && qi < S) {
         const int g = h * p.G + gl_a + w;
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) +
                                               (((int64_t)b * p.Hq + g) * S + qi) * D);
         const uint4* src = reinterpret_cast<const uint4*>(stage + r * D);
 #pragma unroll
@@ -584,7 +581,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // [q * 256 / kc, (q + 1) * 256 / kc) of all of them and writes them out
     __syncthreads();
     cluster_sync_all();
-    if (warp >= 2 && p.out != nullptr) {
+    if (warp >= 2 && out != nullptr) {
       const int t = threadIdx.x - 64;                 // 0..255
       const int rows = 2 * BM / kc;
       const uint32_t stage0 = base + kOffR;
@@ -608,7 +605,7 @@ attn_umma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           v.y = pack_bf16(lo.z, lo.w);
           v.z = pack_bf16(hi.x, hi.y);
           v.w = pack_bf16(hi.z, hi.w);
-          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (((int64_t)b * p.Hq + g) * p.S + qi) * D + d0) = v;
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + (((int64_t)b * p.Hq + g) * p.S + qi) * D + d0) = v;
         }
       }
     }
@@ -650,7 +647,7 @@ int active_clusters(int kc) {
       at[0].val.clusterDim.z = 1;
       cfg.attrs = at;
       cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&n, attn_umma_kernel, &cfg) != cudaSuccess) n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, attn_umma_kernel<1>, &cfg) != cudaSuccess) n = 0;
     }
     cudaGetLastError();
     cache[dev][kc] = n > 0 ? n : -1;
@@ -687,42 +684,53 @@ int split_for(int64_t units, int min_pairs, int forced) {
 
 bool attn_umma_supported(int dtype, int d) { return dtype == kBF16 && d == D; }
 
-cudaError_t launch_attn_umma(const AttnArgs& a, bool pdl, cudaStream_t st) {
-  if (a.d != D) return cudaErrorInvalidValue;
-  cudaError_t e = get_encode();
+namespace {
+
+template <int L>
+cudaError_t launch_group(const AttnArgs* a, int n, bool pdl, cudaStream_t st) {
+  static_assert(sizeof(Group<L>) <= 32000, "kernel parameter space");
+  Group<L> g;
+  memset(&g, 0, sizeof(g));
+  cudaError_t e = cudaSuccess;
+  const int64_t BHq = (int64_t)a[0].B * a[0].Hq, BHkv = (int64_t)a[0].B * a[0].Hkv;
+  const int G = a[0].Hq / a[0].Hkv, n_pg = (G + 1) / 2, n_rt = (int)((a[0].S + BM - 1) / BM);
+  const int64_t units = BHkv * n_pg * n_rt;
+  const int nct = (int)((a[0].n_valid + BN - 1) / BN);
+  const int kc = split_for(units * n, (nct + 2) / 2, a[0].split);   // row tile 0 sees nct + 1 tiles
+  for (int l = 0; l < n; ++l) {
+    const AttnArgs& x = a[l];
+    CUtensorMap* m = g.maps[l];
+    if ((e = make_map(&m[0], x.q, x.S, BHq)) != cudaSuccess) return e;
+    if ((e = make_map(&m[1], x.k, x.S, BHkv)) != cudaSuccess) return e;
+    if ((e = make_map(&m[2], x.v, x.S, BHkv)) != cudaSuccess) return e;
+    // with an empty cache the cache maps are never read; the chunk's stand in
+    const bool has_cache = x.n_valid > 0;
+    if ((e = make_map(&m[3], has_cache ? x.kc : x.k, has_cache ? x.M : x.S, BHkv)) != cudaSuccess) return e;
+    if ((e = make_map(&m[4], has_cache ? x.vc : x.v, has_cache ? x.M : x.S, BHkv)) != cudaSuccess) return e;
+    Params& p = g.p[l];
+    p.colacc = x.colacc;
+    p.err = x.err;
+    p.out = x.out;
+    p.B = x.B;
+    p.Hq = x.Hq;
+    p.Hkv = x.Hkv;
+    p.G = G;
+    p.n_pg = n_pg;
+    p.n_rt = n_rt;
+    p.units = (int)units;
+    p.kc = kc;
+    p.S = x.S;
+    p.M = x.M;
+    p.n_valid = x.n_valid;
+    p.acc_stride = x.acc_stride;
+    p.inject_timeout = x.inject_timeout;
+    p.scale_log2 = x.scale * 1.4426950408889634f;
+    p.fx_scale = fx_scale_of(x.fx_shift);
+  }
+  e = cudaFuncSetAttribute(attn_umma_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  CUtensorMap mq, mk, mv, mkc, mvc;
-  const int64_t BHq = (int64_t)a.B * a.Hq, BHkv = (int64_t)a.B * a.Hkv;
-  if ((e = make_map(&mq, a.q, a.S, BHq)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, a.k, a.S, BHkv)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, a.v, a.S, BHkv)) != cudaSuccess) return e;
-  // with an empty cache the cache maps are never read; the chunk's stand in
-  const bool has_cache = a.n_valid > 0;
-  if ((e = make_map(&mkc, has_cache ? a.kc : a.k, has_cache ? a.M : a.S, BHkv)) != cudaSuccess) return e;
-  if ((e = make_map(&mvc, has_cache ? a.vc : a.v, has_cache ? a.M : a.S, BHkv)) != cudaSuccess) return e;
-  Params p;
-  p.partials = a.partials;
-  p.err = a.err;
-  p.out = a.out;
-  p.B = a.B;
-  p.Hq = a.Hq;
-  p.Hkv = a.Hkv;
-  p.G = a.Hq / a.Hkv;
-  p.n_pg = (p.G + 1) / 2;
-  p.n_rt = (int)((a.S + BM - 1) / BM);
-  p.S = a.S;
-  p.M = a.M;
-  p.n_valid = a.n_valid;
-  p.stride = a.part_stride;
-  p.inject_timeout = a.inject_timeout;
-  p.scale_log2 = a.scale * 1.4426950408889634f;
-  e = cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  const int64_t units = BHkv * p.n_pg * p.n_rt;
-  const int nct = (int)((a.n_valid + BN - 1) / BN);
-  p.kc = split_for(units, (nct + 2) / 2, a.split);   // row tile 0 sees nct + 1 tiles
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(units * p.kc));
+  cfg.gridDim = dim3((unsigned)(units * n * kc));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
@@ -730,12 +738,35 @@ cudaError_t launch_attn_umma(const AttnArgs& a, bool pdl, cudaStream_t st) {
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   at[1].id = cudaLaunchAttributeClusterDimension;
-  at[1].val.clusterDim.x = (unsigned)p.kc;
+  at[1].val.clusterDim.x = (unsigned)kc;
   at[1].val.clusterDim.y = 1;
   at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
-  cfg.numAttrs = p.kc > 1 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, attn_umma_kernel, mq, mk, mv, mkc, mvc, p);
+  cfg.numAttrs = kc > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, attn_umma_kernel<L>, g);
+}
+
+}  // namespace
+
+int attn_umma_max_group() { return kMaxGroup; }
+
+cudaError_t launch_attn_umma_group(const AttnArgs* a, int n, bool pdl, cudaStream_t st) {
+  if (n < 1 || n > kMaxGroup) return cudaErrorInvalidValue;
+  for (int l = 0; l < n; ++l) {
+    const AttnArgs& x = a[l];
+    if (x.d != D) return cudaErrorInvalidValue;
+    // one grid serves layers of identical sizes only
+    if (x.B != a[0].B || x.Hq != a[0].Hq || x.Hkv != a[0].Hkv || x.S != a[0].S || x.M != a[0].M ||
+        x.n_valid != a[0].n_valid || x.fx_shift != a[0].fx_shift || x.split != a[0].split)
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = get_encode();
+  if (e != cudaSuccess) return e;
+  return n == 1 ? launch_group<1>(a, 1, pdl, st) : launch_group<kMaxGroup>(a, n, pdl, st);
+}
+
+cudaError_t launch_attn_umma(const AttnArgs& a, bool pdl, cudaStream_t st) {
+  return launch_attn_umma_group(&a, 1, pdl, st);
 }
 
 }  // namespace h2o

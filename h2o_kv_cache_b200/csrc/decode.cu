@@ -16,8 +16,8 @@
 //   sweep 1: each row's running (max, sum), per warp, then per CTA, then over
 //            the cluster in rank order through distributed shared memory, so
 //            every CTA holds the same log-sum-exp;
-//   sweep 2: p = 2^(s - lse), the key's column sum over all rows (written to
-//            the KV head's single partial row: each key belongs to one CTA),
+//   sweep 2: p = 2^(s - lse), the key's column sum over all rows (added to
+//            the KV head's accumulator row: each key belongs to one CTA),
 //            O += p v per warp; the warps' O are added in warp order, and rank
 //            q adds the CTAs' O of rows r = q (mod kc) in rank order.
 #include "h2o_internal.cuh"
@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
   const T* vb = static_cast<const T*>(a.v) + (int64_t)bh * S * D;
   const T* kcb = static_cast<const T*>(a.kcache) + (int64_t)bh * M * D;
   const T* vcb = static_cast<const T*>(a.vcache) + (int64_t)bh * M * D;
-  float* part = a.partials + (int64_t)bh * a.stride;   // one partial row per KV head
+  unsigned long long* acc = a.colacc + (int64_t)bh * a.acc_stride;   // the KV head's accumulator row
   const int my_r = lane % RM, my_u = lane / RM;   // lane's (row, key in round) after a reduction
   const int my_i = my_r < R ? my_r % (int)S : -1; // its chunk row (causal limit); -1: no such row
 
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
       float cs = p;
 #pragma unroll
       for (int o = 1; o < RM; o <<= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
-      if (my_r == 0 && j < k1) part[j < nv ? j : M + (j - nv)] = cs;
+      if (my_r == 0 && j < k1) colsum_add(acc + (j < nv ? j : M + (j - nv)), cs, a.fx_scale);
 #pragma unroll
       for (int u = 0; u < KR; ++u)
 #pragma unroll

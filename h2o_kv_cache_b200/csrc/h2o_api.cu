@@ -11,6 +11,7 @@
 #include <cstring>
 #include <new>
 #include <string>
+#include <vector>
 
 #include "../../include/h2o.h"
 #include "h2o_internal.cuh"
@@ -47,21 +48,37 @@ struct h2o_ctx {
   void* vc = nullptr;
   float* scores = nullptr;
   int32_t* pos = nullptr;
+  // fixed-point summed weights, [B * Hkv][acc_stride] (cleared by the tail each
+  // step, so zero between steps); acc_stride = 2 M rounded up to a multiple of
+  // 4 holds the M slots and up to M chunk keys
+  unsigned long long* colacc = nullptr;
+  int64_t acc_stride = 0;
   // device error word: mapped pinned host memory, so kernels report into it
   // directly and no copy is enqueued per step; nonzero only after an error
   int* err = nullptr;
-  DevBuf partials, newscore, freed, evicted;
+  DevBuf newscore, freed, evicted;
   // stream-partitioned attention: per-piece row statistics, partial O, unit counters
   DevBuf ws_ml, ws_o, ws_count;
   int n_sm = 0;
   // staging for host pointers
-  DevBuf st_q, st_k, st_v, st_out;
+  // Host inputs are copied on a stream of the handle's own into one of two
+  // staging sets, so the next step's copies overlap this step's kernels: set
+  // s is filled once the kernels of the step that last read it are done
+  // (ev_free[s]), and the caller's stream waits for its copies (ev_in[s]).
+  DevBuf st_q[2], st_k[2], st_v[2], st_out;
+  cudaStream_t copy_st = nullptr;
+  cudaEvent_t ev_in[2] = {}, ev_free[2] = {};
+  bool st_used[2] = {false, false};
+  int st_set = 0;
   cudaEvent_t err_ev = nullptr;   // recorded after each step
   bool err_pending = false;
 
   // fused tail: cluster size for (M, tail_S), 0 = use the three separate kernels
   int64_t tail_S = -1;
   int tail_cs = 0;
+  // the same for grouped steps led by this handle: (S, caches) it was chosen for
+  int64_t grp_tail_S = -1;
+  int grp_tail_n = 0, grp_tail_cs = 0;
 
   // per-kernel timing: a ring of event sets (start, after attention, after the
   // tail), one set per profiled step
@@ -194,9 +211,29 @@ int check_device_error(h2o_ctx* h, bool wait) {
 
 size_t elem_size(int dtype) { return dtype == H2O_F32 ? 4 : 2; }
 
-// Runs one chunk of S tokens (prefill when the cache is empty).
-int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out, int64_t S,
-              cudaStream_t st) {
+// One handle's chunk step between its phases: what prepare_chunk decided and
+// staged, what the launches and finish_chunk use.
+struct ChunkRun {
+  h2o_ctx* h = nullptr;
+  int64_t S = 0, need = 0;
+  size_t q_bytes = 0;
+  const void* dq = nullptr;
+  const void* dk = nullptr;
+  const void* dv = nullptr;
+  void* dout = nullptr;
+  void* out = nullptr;          // the caller's output (host memory when hout)
+  bool hout = false, host_in = false;
+  bool decode = false, stream = false;
+  int fx_shift = 0;
+  h2o::StreamPlan pl;
+  h2o::AttnArgs a;
+  int launches = 0;
+};
+
+// Checks, host-pointer staging, the attention path and the scratch of one
+// chunk of S tokens (prefill when the cache is empty).  Enqueues only copies.
+int prepare_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out, int64_t S,
+                  cudaStream_t st, ChunkRun* r) {
   const int BH = h->B * h->Hkv;
   const size_t es = elem_size(h->dtype);
   const size_t q_bytes = (size_t)h->B * h->Hq * S * h->d * es;
@@ -228,20 +265,34 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   void* dout = out;
   const bool hq = !is_device_ptr(q), hk = !is_device_ptr(k), hv = !is_device_ptr(v);
   const bool hout = out && !is_device_ptr(out);
-  if (hq) {
-    H2O_CUDA(h, ensure(h->st_q, q_bytes), "staging alloc");
-    H2O_CUDA(h, cudaMemcpyAsync(h->st_q.p, q, q_bytes, cudaMemcpyDefault, st), "copy q");
-    dq = h->st_q.p;
-  }
-  if (hk) {
-    H2O_CUDA(h, ensure(h->st_k, kv_bytes), "staging alloc");
-    H2O_CUDA(h, cudaMemcpyAsync(h->st_k.p, k, kv_bytes, cudaMemcpyDefault, st), "copy k");
-    dk = h->st_k.p;
-  }
-  if (hv) {
-    H2O_CUDA(h, ensure(h->st_v, kv_bytes), "staging alloc");
-    H2O_CUDA(h, cudaMemcpyAsync(h->st_v.p, v, kv_bytes, cudaMemcpyDefault, st), "copy v");
-    dv = h->st_v.p;
+  const int set = h->st_set;
+  if (hq || hk || hv) {
+    if (!h->copy_st) {
+      H2O_CUDA(h, cudaStreamCreateWithFlags(&h->copy_st, cudaStreamNonBlocking), "copy stream");
+      for (int i = 0; i < 2; ++i) {
+        H2O_CUDA(h, cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming), "event");
+        H2O_CUDA(h, cudaEventCreateWithFlags(&h->ev_free[i], cudaEventDisableTiming), "event");
+      }
+    }
+    // the step that last read this staging set must be done with it
+    if (h->st_used[set]) H2O_CUDA(h, cudaStreamWaitEvent(h->copy_st, h->ev_free[set], 0), "event wait");
+    if (hq) {
+      H2O_CUDA(h, ensure(h->st_q[set], q_bytes), "staging alloc");
+      H2O_CUDA(h, cudaMemcpyAsync(h->st_q[set].p, q, q_bytes, cudaMemcpyDefault, h->copy_st), "copy q");
+      dq = h->st_q[set].p;
+    }
+    if (hk) {
+      H2O_CUDA(h, ensure(h->st_k[set], kv_bytes), "staging alloc");
+      H2O_CUDA(h, cudaMemcpyAsync(h->st_k[set].p, k, kv_bytes, cudaMemcpyDefault, h->copy_st), "copy k");
+      dk = h->st_k[set].p;
+    }
+    if (hv) {
+      H2O_CUDA(h, ensure(h->st_v[set], kv_bytes), "staging alloc");
+      H2O_CUDA(h, cudaMemcpyAsync(h->st_v[set].p, v, kv_bytes, cudaMemcpyDefault, h->copy_st), "copy v");
+      dv = h->st_v[set].p;
+    }
+    H2O_CUDA(h, cudaEventRecord(h->ev_in[set], h->copy_st), "event");
+    H2O_CUDA(h, cudaStreamWaitEvent(st, h->ev_in[set], 0), "event wait");
   }
   if (hout) {
     H2O_CUDA(h, ensure(h->st_out, q_bytes), "staging alloc");
@@ -249,22 +300,19 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   }
 
   // chunks of a few tokens (G * S <= 16 rows per KV head, and a cache whose
-  // scores fit the decode kernel's shared memory) take the decode kernel, which
-  // writes one partial row per KV head; forcing a tensor-core path
-  // (H2O_ATTN_MODE) bypasses it
+  // scores fit the decode kernel's shared memory) take the decode kernel;
+  // forcing a tensor-core path (H2O_ATTN_MODE) bypasses it
   const bool decode = h2o::decode_supported(h->G, S, h->n_valid + S) && attn_mode() == 0;
-  // scratch sized for this chunk
-  const int row_tile = decode ? (int)S : h->row_tile;
-  const int n_rt = decode ? 1 : (int)((S + h->row_tile - 1) / h->row_tile);
-  const int64_t stride = h2o::partial_stride(h->M, S);
+  const int fx_shift = h2o::colsum_shift(S, h->G);
 
-  h2o::AttnArgs a;
+  h2o::AttnArgs& a = r->a;
   a.q = dq;
   a.k = dk;
   a.v = dv;
   a.out = dout;
   a.kc = h->kc;
   a.vc = h->vc;
+  a.colacc = h->colacc;
   a.err = h->err;
   a.B = h->B;
   a.Hq = h->Hq;
@@ -273,7 +321,8 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   a.S = S;
   a.M = h->M;
   a.n_valid = h->n_valid;
-  a.part_stride = stride;
+  a.acc_stride = h->acc_stride;
+  a.fx_shift = fx_shift;
   a.split = attn_split();
   a.inject_timeout = inject_timeout() ? 1 : 0;
   a.scale = (float)(1.0 / std::sqrt((double)h->d));
@@ -283,132 +332,261 @@ int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out
   // pays when the one-kernel grid would leave SMs idle (n_sm / 2 .. 2 n_sm
   // units) and units are long enough (>= 24 pairs on average) for a piece
   // boundary's Q reload and epilogue.
-  h2o::StreamPlan pl;
   bool stream = false;
   if (!decode && h->use_umma) {
     if (h->n_sm == 0) H2O_CUDA(h, cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device),
                                "device attribute");
     const int mode = attn_mode();
-    if (mode != 1 && (!a.inject_timeout || mode == 2) && h2o::attn_stream_plan(a, h->n_sm, &pl))
-      stream = mode == 2 || (2 * pl.units >= h->n_sm && pl.units <= 2 * h->n_sm &&
-                             pl.total_pairs >= 24 * (int64_t)pl.units);
+    if (mode != 1 && (!a.inject_timeout || mode == 2) && h2o::attn_stream_plan(a, h->n_sm, &r->pl))
+      stream = mode == 2 || (2 * r->pl.units >= h->n_sm && r->pl.units <= 2 * h->n_sm &&
+                             r->pl.total_pairs >= 24 * (int64_t)r->pl.units);
   }
-  const int n_grp = decode ? 1 : stream ? h2o::stream_partial_groups(h->G)
-                                        : h2o::partial_groups(h->G, h->use_umma);
-  const size_t part_bytes = (size_t)BH * n_grp * n_rt * stride * sizeof(float);
-  H2O_CUDA(h, ensure(h->partials, part_bytes), "scratch alloc");
-  a.partials = static_cast<float*>(h->partials.p);
   H2O_CUDA(h, ensure(h->freed, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
   H2O_CUDA(h, ensure(h->evicted, (size_t)BH * S * sizeof(int32_t)), "scratch alloc");
+  if (stream) {
+    H2O_CUDA(h, ensure(h->ws_ml, r->pl.ml_bytes), "scratch alloc");
+    if (r->pl.o_bytes) H2O_CUDA(h, ensure(h->ws_o, r->pl.o_bytes), "scratch alloc");
+    H2O_CUDA(h, ensure(h->ws_count, r->pl.count_bytes), "scratch alloc");
+  }
+  if (S != h->tail_S) {
+    h->tail_cs = split_tail() ? 0 : h2o::tail_cluster_size(h->M, S, BH);
+    h->tail_S = S;
+  }
+  if (h->tail_cs == 0) H2O_CUDA(h, ensure(h->newscore, (size_t)BH * S * sizeof(float)), "scratch alloc");
 
-  cudaEvent_t* evs = h->ev[h->prof_steps % h2o_ctx::kProfRing];
-  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[0], st), "event");
+  r->h = h;
+  r->S = S;
+  r->need = need;
+  r->q_bytes = q_bytes;
+  r->dq = dq;
+  r->dk = dk;
+  r->dv = dv;
+  r->dout = dout;
+  r->out = out;
+  r->hout = hout;
+  r->host_in = hq || hk || hv;
+  r->decode = decode;
+  r->stream = stream;
+  r->fx_shift = fx_shift;
+  r->launches = 0;
+  return H2O_OK;
+}
 
+// The attention launch(es) of one prepared chunk.
+int launch_attention(ChunkRun& r, cudaStream_t st) {
+  h2o_ctx* h = r.h;
+  const int BH = h->B * h->Hkv;
   if (fault_injected("launch")) return fail(h, H2O_ECUDA, "injected launch failure");
   cudaError_t e = cudaSuccess;
-  int launches = 1;
-  if (decode) {
+  if (r.decode) {
     h2o::DecodeArgs da;
-    da.q = dq;
-    da.k = dk;
-    da.v = dv;
-    da.out = dout;
+    da.q = r.dq;
+    da.k = r.dk;
+    da.v = r.dv;
+    da.out = r.dout;
     da.kcache = h->kc;
     da.vcache = h->vc;
-    da.partials = static_cast<float*>(h->partials.p);
+    da.colacc = h->colacc;
     da.err = h->err;
     da.B = h->B;
     da.Hq = h->Hq;
     da.Hkv = h->Hkv;
     da.G = h->G;
     da.d = h->d;
-    da.S = S;
+    da.S = r.S;
     da.M = h->M;
     da.n_valid = h->n_valid;
-    da.stride = stride;
-    da.scale_log2 = a.scale * 1.4426950408889634f;
+    da.acc_stride = h->acc_stride;
+    da.scale_log2 = r.a.scale * 1.4426950408889634f;
+    da.fx_scale = h2o::fx_scale_of(r.fx_shift);
     e = h2o::launch_decode(da, h->dtype, BH, true, st);
+    r.launches += 1;
   } else if (h->use_umma) {
-    if (stream) {
-      H2O_CUDA(h, ensure(h->ws_ml, pl.ml_bytes), "scratch alloc");
-      if (pl.o_bytes) H2O_CUDA(h, ensure(h->ws_o, pl.o_bytes), "scratch alloc");
-      H2O_CUDA(h, ensure(h->ws_count, pl.count_bytes), "scratch alloc");
-      e = h2o::launch_attn_stream(a, pl, h->ws_ml.p, h->ws_o.p, static_cast<int*>(h->ws_count.p), true, st);
-      launches = 2;
+    if (r.stream) {
+      e = h2o::launch_attn_stream(r.a, r.pl, h->ws_ml.p, h->ws_o.p, static_cast<int*>(h->ws_count.p),
+                                  true, st);
+      r.launches += 2;
     } else {
-      e = h2o::launch_attn_umma(a, true, st);
+      e = h2o::launch_attn_umma(r.a, true, st);
+      r.launches += 1;
     }
   } else {
-    e = h2o::launch_attn_simt(a, h->dtype, true, st);
+    e = h2o::launch_attn_simt(r.a, h->dtype, true, st);
+    r.launches += 1;
   }
   if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
-  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[1], st), "event");
+  return H2O_OK;
+}
 
-  if (S != h->tail_S) {
-    h->tail_cs = split_tail() ? 0 : h2o::tail_cluster_size(h->M, S, BH);
-    h->tail_S = S;
-  }
+h2o::TailArgs tail_args(const ChunkRun& r) {
+  const h2o_ctx* h = r.h;
+  h2o::TailArgs t;
+  t.colacc = h->colacc;
+  t.scores = h->scores;
+  t.pos = h->pos;
+  t.k = static_cast<const uint4*>(r.dk);
+  t.v = static_cast<const uint4*>(r.dv);
+  t.kc = static_cast<uint4*>(h->kc);
+  t.vc = static_cast<uint4*>(h->vc);
+  t.freed = static_cast<int32_t*>(h->freed.p);
+  t.evicted = static_cast<int32_t*>(h->evicted.p);
+  t.err = h->err;
+  t.M = h->M;
+  t.S = r.S;
+  t.n_valid = h->n_valid;
+  t.t0 = h->t0;
+  t.R = h->R;
+  t.need = r.need;
+  t.acc_stride = h->acc_stride;
+  t.fx_inv = h2o::fx_inv_of(r.fx_shift);
+  t.row_vecs = (int)(h->d * elem_size(h->dtype) / 16);
+  t.per = t.per_s = 0;
+  return t;
+}
+
+// Score accumulate + select + scatter of one prepared chunk.
+int launch_tail(ChunkRun& r, cudaStream_t st) {
+  h2o_ctx* h = r.h;
+  const int BH = h->B * h->Hkv;
+  cudaError_t e = cudaSuccess;
   if (h->tail_cs > 0) {
-    h2o::TailArgs t;
-    t.partials = static_cast<const float*>(h->partials.p);
-    t.scores = h->scores;
-    t.pos = h->pos;
-    t.k = static_cast<const uint4*>(dk);
-    t.v = static_cast<const uint4*>(dv);
-    t.kc = static_cast<uint4*>(h->kc);
-    t.vc = static_cast<uint4*>(h->vc);
-    t.freed = static_cast<int32_t*>(h->freed.p);
-    t.evicted = static_cast<int32_t*>(h->evicted.p);
-    t.err = h->err;
-    t.M = h->M;
-    t.S = S;
-    t.n_valid = h->n_valid;
-    t.t0 = h->t0;
-    t.R = h->R;
-    t.need = need;
-    t.stride = stride;
-    t.n_grp = n_grp;
-    t.n_rt = n_rt;
-    t.row_tile = row_tile;
-    t.row_vecs = (int)(h->d * es / 16);
-    e = h2o::launch_tail(t, BH, h->tail_cs, true, st);
+    e = h2o::launch_tail(tail_args(r), BH, h->tail_cs, true, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "tail launch");
-    h->last_launches = launches + 1;
+    r.launches += 1;
   } else {
-    H2O_CUDA(h, ensure(h->newscore, (size_t)BH * S * sizeof(float)), "scratch alloc");
-    e = h2o::launch_score_reduce(static_cast<float*>(h->partials.p), h->scores,
-                                 static_cast<float*>(h->newscore.p), BH, n_grp, S, h->M,
-                                 h->n_valid, row_tile, stride, st);
+    e = h2o::launch_score_reduce(h->colacc, h->acc_stride, h2o::fx_inv_of(r.fx_shift), h->scores,
+                                 static_cast<float*>(h->newscore.p), BH, r.S, h->M, h->n_valid, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "score reduce launch");
-    e = h2o::launch_select(h->scores, h->pos, BH, h->M, h->t0, h->R, need, h->n_valid, S,
-                           static_cast<int32_t*>(h->freed.p), S, h->err, st);
+    e = h2o::launch_select(h->scores, h->pos, BH, h->M, h->t0, h->R, r.need, h->n_valid, r.S,
+                           static_cast<int32_t*>(h->freed.p), r.S, h->err, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "select launch");
-    e = h2o::launch_scatter(dk, dv, h->kc, h->vc, h->scores, h->pos,
+    e = h2o::launch_scatter(r.dk, r.dv, h->kc, h->vc, h->scores, h->pos,
                             static_cast<int32_t*>(h->freed.p), static_cast<float*>(h->newscore.p),
-                            static_cast<int32_t*>(h->evicted.p), BH, S, h->M, h->d, (int)es, h->t0,
-                            st);
+                            static_cast<int32_t*>(h->evicted.p), BH, r.S, h->M, h->d,
+                            (int)elem_size(h->dtype), h->t0, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "scatter launch");
-    h->last_launches = launches + 3;
+    r.launches += 3;
   }
+  return H2O_OK;
+}
+
+// After the launches: the output copy for host buffers, the staging set's
+// release, the error event, the counters; with H2O_SYNC_CHECK=1 the step's own
+// device error is waited for and reported.
+int finish_chunk(ChunkRun& r, cudaStream_t st) {
+  h2o_ctx* h = r.h;
+  if (r.host_in) {
+    const int set = h->st_set;
+    H2O_CUDA(h, cudaEventRecord(h->ev_free[set], st), "event");
+    h->st_used[set] = true;
+    h->st_set = set ^ 1;
+  }
+  if (r.hout) H2O_CUDA(h, cudaMemcpyAsync(r.out, r.dout, r.q_bytes, cudaMemcpyDefault, st), "copy out");
+  // the error word is read once this event has completed (by the next call)
+  H2O_CUDA(h, cudaEventRecord(h->err_ev, st), "event");
+  h->err_pending = true;
+  h->t0 += r.S;
+  h->n_valid = h->n_valid + r.S < h->M ? h->n_valid + r.S : h->M;
+  h->last_S = r.S;
+  h->last_launches = r.launches;
+  if (sync_check_enabled()) return check_device_error(h, true);
+  return H2O_OK;
+}
+
+// Runs one chunk of S tokens (prefill when the cache is empty).
+int run_chunk(h2o_ctx* h, const void* q, const void* k, const void* v, void* out, int64_t S,
+              cudaStream_t st) {
+  ChunkRun r;
+  int rc = prepare_chunk(h, q, k, v, out, S, st, &r);
+  if (rc != H2O_OK) return rc;
+  cudaEvent_t* evs = h->ev[h->prof_steps % h2o_ctx::kProfRing];
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[0], st), "event");
+  if ((rc = launch_attention(r, st)) != H2O_OK) return rc;
+  if (h->prof) H2O_CUDA(h, cudaEventRecord(evs[1], st), "event");
+  if ((rc = launch_tail(r, st)) != H2O_OK) return rc;
   if (h->prof) {
     H2O_CUDA(h, cudaEventRecord(evs[2], st), "event");
     ++h->prof_steps;
   }
+  return finish_chunk(r, st);
+}
 
-  if (hout) H2O_CUDA(h, cudaMemcpyAsync(out, dout, q_bytes, cudaMemcpyDefault, st), "copy out");
-
-  // the error word is read once this event has completed (by the next call)
-  H2O_CUDA(h, cudaEventRecord(h->err_ev, st), "event");
-  h->err_pending = true;
-
-  h->t0 += S;
-  h->n_valid = h->n_valid + S < h->M ? h->n_valid + S : h->M;
-  h->last_S = S;
-  if (hq || hk || hv || hout || sync_check_enabled()) {
-    rc = check_device_error(h, true);
-    if (rc != H2O_OK) return rc;
+// Several layers' chunk steps.  Layers of identical sizes on the one-kernel
+// tensor-core path share one attention grid and one tail grid (in groups of up
+// to the kernels' maximum); any other layer runs its own step.
+int run_layers(h2o_ctx** hs, int n, const void* const* q, const void* const* k,
+               const void* const* v, void* const* out, int64_t S, cudaStream_t st) {
+  std::vector<ChunkRun> runs((size_t)n);
+  for (int l = 0; l < n; ++l) {
+    int rc = prepare_chunk(hs[l], q[l], k[l], v[l], out ? out[l] : nullptr, S, st, &runs[(size_t)l]);
+    if (rc != H2O_OK) {
+      // the layers before l are staged but not launched: nothing changed yet
+      if (l > 0) fail(hs[0], rc, "layer %d: %s", l, hs[l]->msg.c_str());
+      return rc;
+    }
   }
-  return H2O_OK;
+  h2o_ctx* h0 = hs[0];
+  auto groupable = [&](const ChunkRun& r) {
+    const h2o_ctx* h = r.h;
+    return h->use_umma && !r.decode && !r.stream && h->tail_cs > 0 && h->device == h0->device &&
+           h->B == h0->B && h->Hq == h0->Hq && h->Hkv == h0->Hkv && h->d == h0->d &&
+           h->M == h0->M && h->R == h0->R && h->t0 == h0->t0 && h->n_valid == h0->n_valid &&
+           h->tail_cs == h0->tail_cs && r.a.split == runs[0].a.split &&
+           r.a.inject_timeout == runs[0].a.inject_timeout;
+  };
+  bool all = true;
+  for (int l = 0; l < n; ++l) all = all && groupable(runs[(size_t)l]);
+  cudaEvent_t* evs = h0->ev[h0->prof_steps % h2o_ctx::kProfRing];
+  const bool prof = h0->prof;
+  if (prof) H2O_CUDA(h0, cudaEventRecord(evs[0], st), "event");
+  int rc = H2O_OK;
+  if (!all) {
+    // layer after layer, each with its own launches
+    for (int l = 0; l < n && rc == H2O_OK; ++l) rc = launch_attention(runs[(size_t)l], st);
+    if (prof && rc == H2O_OK) H2O_CUDA(h0, cudaEventRecord(evs[1], st), "event");
+    for (int l = 0; l < n && rc == H2O_OK; ++l) rc = launch_tail(runs[(size_t)l], st);
+  } else {
+    if (fault_injected("launch")) return fail(h0, H2O_ECUDA, "injected launch failure");
+    const int BH = h0->B * h0->Hkv;
+    const int ga = h2o::attn_umma_max_group(), gt = h2o::tail_max_group();
+    std::vector<h2o::AttnArgs> aa((size_t)n);
+    std::vector<h2o::TailArgs> ta((size_t)n);
+    for (int l = 0; l < n; ++l) {
+      aa[(size_t)l] = runs[(size_t)l].a;
+      ta[(size_t)l] = tail_args(runs[(size_t)l]);
+    }
+    for (int l0 = 0; l0 < n; l0 += ga) {
+      const int m = n - l0 < ga ? n - l0 : ga;
+      cudaError_t e = h2o::launch_attn_umma_group(aa.data() + l0, m, true, st);
+      if (e != cudaSuccess) return cuda_fail(h0, e, "grouped attention launch");
+      runs[(size_t)l0].launches += 1;
+    }
+    if (prof) H2O_CUDA(h0, cudaEventRecord(evs[1], st), "event");
+    if (h0->grp_tail_S != S || h0->grp_tail_n != n) {
+      const int m = n < gt ? n : gt;
+      h0->grp_tail_cs = m > 1 ? h2o::tail_cluster_size(h0->M, S, m * BH, true) : h0->tail_cs;
+      h0->grp_tail_S = S;
+      h0->grp_tail_n = n;
+    }
+    for (int l0 = 0; l0 < n; l0 += gt) {
+      const int m = n - l0 < gt ? n - l0 : gt;
+      const int cs = m > 1 ? h0->grp_tail_cs : h0->tail_cs;
+      if (cs < 1) return fail(h0, H2O_ECUDA, "grouped tail: no cluster size fits");
+      cudaError_t e = h2o::launch_tail_group(ta.data() + l0, m, BH, cs, true, st);
+      if (e != cudaSuccess) return cuda_fail(h0, e, "grouped tail launch");
+      runs[(size_t)l0].launches += 1;
+    }
+  }
+  if (rc != H2O_OK) return rc;
+  if (prof) {
+    H2O_CUDA(h0, cudaEventRecord(evs[2], st), "event");
+    ++h0->prof_steps;
+  }
+  for (int l = 0; l < n; ++l) {
+    const int r2 = finish_chunk(runs[(size_t)l], st);
+    if (r2 != H2O_OK && rc == H2O_OK) rc = r2;
+  }
+  return rc;
 }
 
 // Frees the per-handle device state (cache, scores, positions, error word,
@@ -418,6 +596,7 @@ void release_state(h2o_ctx* h) {
   cudaFree(h->vc);
   cudaFree(h->scores);
   cudaFree(h->pos);
+  cudaFree(h->colacc);
   if (h->err) cudaFreeHost(h->err);
   if (h->err_ev) cudaEventDestroy(h->err_ev);
   for (auto& set : h->ev)
@@ -428,6 +607,7 @@ void release_state(h2o_ctx* h) {
   h->kc = h->vc = nullptr;
   h->scores = nullptr;
   h->pos = nullptr;
+  h->colacc = nullptr;
   h->err = nullptr;
   h->err_ev = nullptr;
   h->device = -1;
@@ -444,6 +624,9 @@ int alloc_state_impl(h2o_ctx* h, int B) {
   H2O_CUDA(h, dev_alloc(&h->vc, slots * h->d * es), "cache alloc");
   H2O_CUDA(h, dev_alloc((void**)&h->scores, slots * sizeof(float)), "state alloc");
   H2O_CUDA(h, dev_alloc((void**)&h->pos, slots * sizeof(int32_t)), "state alloc");
+  h->acc_stride = (2 * h->M + 3) & ~(int64_t)3;
+  const size_t acc_bytes = (size_t)B * h->Hkv * h->acc_stride * sizeof(unsigned long long);
+  H2O_CUDA(h, dev_alloc((void**)&h->colacc, acc_bytes), "state alloc");
   {
     void* hp = nullptr;
     H2O_CUDA(h, cudaHostAlloc(&hp, sizeof(int), cudaHostAllocMapped), "pinned alloc");
@@ -454,6 +637,7 @@ int alloc_state_impl(h2o_ctx* h, int B) {
   H2O_CUDA(h, cudaMemset(h->vc, 0, slots * h->d * es), "memset");
   H2O_CUDA(h, cudaMemset(h->scores, 0, slots * sizeof(float)), "memset");
   H2O_CUDA(h, cudaMemset(h->pos, 0xFF, slots * sizeof(int32_t)), "memset");
+  H2O_CUDA(h, cudaMemset(h->colacc, 0, acc_bytes), "memset");
   H2O_CUDA(h, cudaEventCreateWithFlags(&h->err_ev, cudaEventDisableTiming), "event");
   for (auto& set : h->ev)
     for (auto& ev : set) H2O_CUDA(h, cudaEventCreate(&ev), "event");
@@ -527,6 +711,26 @@ int h2o_step(h2o_t h, const void* q, const void* k, const void* v, void* out, in
     return fail(h, H2O_ESHAPE, "h2o_step: S=%lld exceeds the cache capacity M=%lld",
                 (long long)S, (long long)h->M);
   return run_chunk(h, q, k, v, out, S, static_cast<cudaStream_t>(stream));
+}
+
+int h2o_step_layers(h2o_t* hs, int n, const void* const* q, const void* const* k,
+                    const void* const* v, void* const* out, int64_t S, void* stream) {
+  if (!hs || n < 1) return fail(nullptr, H2O_EINVAL, "h2o_step_layers: need n >= 1 handles");
+  if (!q || !k || !v) return fail(nullptr, H2O_EINVAL, "h2o_step_layers: q, k and v arrays must not be NULL");
+  for (int l = 0; l < n; ++l) {
+    h2o_ctx* h = hs[l];
+    if (!h) return fail(nullptr, H2O_EINVAL, "h2o_step_layers: handle %d is NULL", l);
+    for (int j = 0; j < l; ++j)
+      if (hs[j] == h) return fail(h, H2O_EINVAL, "h2o_step_layers: handle %d repeats handle %d", l, j);
+    if (!h->prefilled) return fail(h, H2O_ESTATE, "h2o_step_layers: handle %d not prefilled", l);
+    if (!q[l] || !k[l] || !v[l])
+      return fail(h, H2O_EINVAL, "h2o_step_layers: q, k and v of layer %d must not be NULL", l);
+    if (S < 1) return fail(h, H2O_EINVAL, "h2o_step_layers: need S >= 1");
+    if (S > h->M)
+      return fail(h, H2O_ESHAPE, "h2o_step_layers: S=%lld exceeds the cache capacity M=%lld of layer %d",
+                  (long long)S, (long long)h->M, l);
+  }
+  return run_layers(hs, n, q, k, v, out, S, static_cast<cudaStream_t>(stream));
 }
 
 int h2o_read_state(h2o_t h, int32_t* slots, float* scores, int32_t* positions, void* stream) {
@@ -622,9 +826,15 @@ int h2o_destroy(h2o_t h) {
     cudaSetDevice(h->device);
     cudaDeviceSynchronize();
   }
-  for (DevBuf* b : {&h->partials, &h->newscore, &h->freed, &h->evicted, &h->ws_ml, &h->ws_o,
-                    &h->ws_count, &h->st_q, &h->st_k, &h->st_v, &h->st_out})
+  for (DevBuf* b : {&h->newscore, &h->freed, &h->evicted, &h->ws_ml, &h->ws_o,
+                    &h->ws_count, &h->st_q[0], &h->st_k[0], &h->st_v[0], &h->st_q[1], &h->st_k[1],
+                    &h->st_v[1], &h->st_out})
     cudaFree(b->p);
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_free[i]) cudaEventDestroy(h->ev_free[i]);
+  }
+  if (h->copy_st) cudaStreamDestroy(h->copy_st);
   release_state(h);
   delete h;
   return H2O_OK;

@@ -4,9 +4,9 @@
 // all of the GPU's memory for its own pool up front has none left to give, and
 // latency-critical code cannot afford cudaMalloc's implicit device
 // synchronisation.  This entry point therefore takes every input and output
-// from the caller and keeps its only scratch -- the per-row-tile partial column
-// sums and the device error word -- in a fixed-size array defined here at file
-// scope.  Each GPU that loads the library holds that array until the process
+// from the caller and keeps its only scratch -- the fixed-point accumulator
+// rows of the summed weights and the device error word -- in a fixed-size
+// array defined here at file scope.  Each GPU that loads the library holds that array until the process
 // exits.
 #include <cuda_runtime.h>
 
@@ -19,9 +19,10 @@
 
 namespace {
 
-// 16 MiB: 4 Mi floats of partial column sums, then the error word.
-constexpr size_t kScratchFloats = (size_t)4 << 20;
-constexpr size_t kScratchBytes = kScratchFloats * sizeof(float) + 256;
+// 16 MiB: 2 Mi 64-bit accumulator words (one row of M + S per (b, KV head)),
+// then the error word.
+constexpr size_t kScratchWords = (size_t)2 << 20;
+constexpr size_t kScratchBytes = kScratchWords * sizeof(unsigned long long) + 256;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
@@ -55,27 +56,14 @@ cudaError_t scratch_address(void** out) {
 }
 
 // colsum[bh, c] for c < M: the slot's summed weight (0 for slots >= n_valid);
-// colsum[bh, M + j]: chunk key j's summed weight.  Fixed-order sums of the
-// attention kernel's partial rows.
-__global__ void colsum_kernel(const float* __restrict__ partials, float* __restrict__ colsum, int G,
-                              int64_t S, int64_t M, int64_t n_valid, int row_tile, int64_t stride) {
+// colsum[bh, M + j]: chunk key j's summed weight; from the accumulator rows.
+__global__ void colsum_kernel(const unsigned long long* __restrict__ acc, float* __restrict__ colsum,
+                              int64_t S, int64_t M, int64_t stride, float fx_inv) {
   const int bh = blockIdx.y;
   const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t ncol = M + S;
   if (c >= ncol) return;
-  const int n_rt = (int)((S + row_tile - 1) / row_tile);
-  const float* base = partials + (int64_t)bh * (G * n_rt) * stride;
-  float acc = 0.f;
-  if (c < M) {
-    if (c < n_valid)
-      for (int t = 0; t < G * n_rt; ++t) acc += base[(int64_t)t * stride + c];
-  } else {
-    const int64_t j = c - M;
-    const int rt0 = (int)(j / row_tile);
-    for (int gl = 0; gl < G; ++gl)
-      for (int rt = rt0; rt < n_rt; ++rt) acc += base[(int64_t)(gl * n_rt + rt) * stride + c];
-  }
-  colsum[(int64_t)bh * ncol + c] = acc;
+  colsum[(int64_t)bh * ncol + c] = h2o::colsum_value(acc[(int64_t)bh * stride + c], fx_inv);
 }
 
 }  // namespace
@@ -90,29 +78,29 @@ extern "C" int h2o_attend_noalloc(const void* q, const void* k, const void* v, c
       (dtype != H2O_F32 && dtype != H2O_BF16) || S < 1 || M < 0 || n_valid < 0 || n_valid > M)
     return set_err(H2O_EINVAL, "bad sizes");
   const bool umma = h2o::attn_umma_supported(dtype, d);
-  const int row_tile = umma ? h2o::kUmmaRowTile : h2o::kSimtRowTile;
   const int G = Hq / Hkv;
-  const int64_t n_rt = (S + row_tile - 1) / row_tile;
-  const int64_t stride = h2o::partial_stride(M, S);
-  const double need = (double)B * Hkv * G * n_rt * (double)stride;
-  if (need > (double)kScratchFloats) {
+  const int64_t stride = (M + S + 3) & ~(int64_t)3;   // accumulator words per (b, KV head)
+  const double need = (double)B * Hkv * (double)stride;
+  if (need > (double)kScratchWords) {
     char msg[256];
     snprintf(msg, sizeof(msg),
-             "problem needs %.0f scratch floats, above the fixed maximum of %zu "
-             "(B*Hkv*(Hq/Hkv)*ceil(S/%d)*(M+S rounded up to a multiple of 4) must be <= %zu)",
-             need, kScratchFloats, row_tile, kScratchFloats);
+             "problem needs %.0f scratch words, above the fixed maximum of %zu "
+             "(B*Hkv*(M+S rounded up to a multiple of 4) must be <= %zu)",
+             need, kScratchWords, kScratchWords);
     return set_err(H2O_ESHAPE, msg);
   }
   void* base = nullptr;
   cudaError_t e = scratch_address(&base);
   if (e != cudaSuccess) return set_err(H2O_ECUDA, cudaGetErrorString(e));
-  float* partials = static_cast<float*>(base);
-  int* err = reinterpret_cast<int*>(static_cast<unsigned char*>(base) + kScratchFloats * sizeof(float));
+  unsigned long long* acc = static_cast<unsigned long long*>(base);
+  int* err = reinterpret_cast<int*>(static_cast<unsigned char*>(base) +
+                                    kScratchWords * sizeof(unsigned long long));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  // The error word must start at zero; the partials need no clearing (the
-  // column sums read only entries the attention kernel wrote in this call).
-  e = cudaMemsetAsync(err, 0, sizeof(int), st);
+  // The accumulator rows and the error word must start at zero: the array
+  // keeps whatever the previous call left.
+  e = cudaMemsetAsync(acc, 0, (size_t)need * sizeof(unsigned long long), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(err, 0, sizeof(int), st);
   if (e != cudaSuccess) return set_err(H2O_ECUDA, cudaGetErrorString(e));
 
   h2o::AttnArgs a;
@@ -122,7 +110,7 @@ extern "C" int h2o_attend_noalloc(const void* q, const void* k, const void* v, c
   a.out = out;
   a.kc = k_cache;
   a.vc = v_cache;
-  a.partials = partials;
+  a.colacc = acc;
   a.err = err;
   a.B = B;
   a.Hq = Hq;
@@ -131,14 +119,14 @@ extern "C" int h2o_attend_noalloc(const void* q, const void* k, const void* v, c
   a.S = S;
   a.M = M;
   a.n_valid = n_valid;
-  a.part_stride = stride;
+  a.acc_stride = stride;
   a.scale = (float)(1.0 / std::sqrt((double)d));
+  a.fx_shift = h2o::colsum_shift(S, G);
   e = umma ? h2o::launch_attn_umma(a, false, st) : h2o::launch_attn_simt(a, dtype, false, st);
   if (e != cudaSuccess) return set_err(H2O_ECUDA, cudaGetErrorString(e));
   const int threads = 256;
   dim3 grid((unsigned)((M + S + threads - 1) / threads), (unsigned)(B * Hkv));
-  colsum_kernel<<<grid, threads, 0, st>>>(partials, colsum, h2o::partial_groups(G, umma), S, M,
-                                           n_valid, row_tile, stride);
+  colsum_kernel<<<grid, threads, 0, st>>>(acc, colsum, S, M, stride, h2o::fx_inv_of(a.fx_shift));
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_err(H2O_ECUDA, cudaGetErrorString(e));
   return H2O_OK;

@@ -12,46 +12,22 @@ namespace h2o {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Score accumulation: fixed-order sum of the attention kernel's partial rows.
+// Score accumulation: each column's summed weight from the fixed-point
+// accumulator row (the word is cleared for the next chunk).
 // ---------------------------------------------------------------------------
-__global__ void score_reduce_kernel(const float* __restrict__ partials, float* __restrict__ scores,
-                                    float* __restrict__ newscore, int G, int64_t S, int64_t M,
-                                    int64_t n_valid, int row_tile, int64_t ncol) {
+__global__ void score_reduce_kernel(unsigned long long* __restrict__ colacc, int64_t acc_stride,
+                                    float fx_inv, float* __restrict__ scores,
+                                    float* __restrict__ newscore, int64_t S, int64_t M,
+                                    int64_t n_valid) {
   const int bh = blockIdx.y;
   const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= n_valid + S) return;
-  const int n_rt = (int)((S + row_tile - 1) / row_tile);
-  const float* base = partials + (int64_t)bh * (G * n_rt) * ncol;
-  float run[kQuarters];
-  if (c < n_valid) {
-    const int n = G * n_rt;
-#pragma unroll
-    for (int q = 0; q < kQuarters; ++q) {
-      run[q] = 0.f;
-      for (int t = q * n / kQuarters; t < (q + 1) * n / kQuarters; ++t) run[q] += base[(int64_t)t * ncol + c];
-    }
-    float acc = run[0];
-#pragma unroll
-    for (int q = 1; q < kQuarters; ++q) acc += run[q];
-    scores[(int64_t)bh * M + c] += acc;
-  } else {
-    const int64_t j = c - n_valid;
-    const int rt0 = (int)(j / row_tile);       // first row tile that sees chunk key j
-    const int span = n_rt - rt0;
-    const int n = G * span;                    // rows (gl, rt >= rt0), gl-major
-#pragma unroll
-    for (int q = 0; q < kQuarters; ++q) {
-      run[q] = 0.f;
-      for (int t = q * n / kQuarters; t < (q + 1) * n / kQuarters; ++t) {
-        const int gl = t / span, rt = rt0 + t - gl * span;
-        run[q] += base[(int64_t)(gl * n_rt + rt) * ncol + M + j];
-      }
-    }
-    float acc = run[0];
-#pragma unroll
-    for (int q = 1; q < kQuarters; ++q) acc += run[q];
-    newscore[(int64_t)bh * S + j] = acc;
-  }
+  unsigned long long* acc = colacc + (int64_t)bh * acc_stride;
+  const int64_t col = c < n_valid ? c : M + (c - n_valid);
+  const float v = colsum_value(acc[col], fx_inv);
+  acc[col] = 0ull;
+  if (c < n_valid) scores[(int64_t)bh * M + c] += v;
+  else newscore[(int64_t)bh * S + (c - n_valid)] = v;
 }
 
 // ---------------------------------------------------------------------------
@@ -213,13 +189,13 @@ __global__ void scatter_kernel(const uint4* __restrict__ k, const uint4* __restr
 
 }  // namespace
 
-cudaError_t launch_score_reduce(const float* partials, float* scores, float* newscore, int BH,
-                                int G, int64_t S, int64_t M, int64_t n_valid, int row_tile,
-                                int64_t part_stride, cudaStream_t st) {
+cudaError_t launch_score_reduce(unsigned long long* colacc, int64_t acc_stride, float fx_inv,
+                                float* scores, float* newscore, int BH, int64_t S, int64_t M,
+                                int64_t n_valid, cudaStream_t st) {
   const int threads = 256;
   dim3 grid((unsigned)((n_valid + S + threads - 1) / threads), (unsigned)BH);
-  score_reduce_kernel<<<grid, threads, 0, st>>>(partials, scores, newscore, G, S, M, n_valid,
-                                                row_tile, part_stride);
+  score_reduce_kernel<<<grid, threads, 0, st>>>(colacc, acc_stride, fx_inv, scores, newscore, S, M,
+                                                n_valid);
   return cudaGetLastError();
 }
 

@@ -10,11 +10,11 @@
 // One thread-block cluster per (b, KV head); CTA `rank` of the cluster owns
 // cache slots [rank * per, (rank + 1) * per) and chunk rows
 // [rank * per_s, (rank + 1) * per_s).  Phases, separated by cluster barriers:
-//   1. add the partial rows of the summed weights to the scores of its slots
-//      (fixed row order, so the result does not depend on scheduling), and
+//   1. add the summed weights (the fixed-point accumulator row the attention
+//      kernel filled, read once and cleared) to the scores of its slots, and
 //      form each eligible slot's 64-bit key (order-preserving score bits,
-//      token position) in shared memory; reduce the chunk columns of its rows
-//      into the new tokens' initial scores;
+//      token position) in shared memory; the chunk keys' summed weights are
+//      the new tokens' initial scores;
 //   2. MSD radix select, 11 bits a pass: every CTA adds its digit counts into
 //      rank 0's histogram through distributed shared memory, then all CTAs
 //      read the merged histogram and take the same decision;
@@ -24,6 +24,7 @@
 //      at the start, so only the stores remain here), recording the position
 //      each slot held before: with the freed list, the chunk's buffer delta.
 #include <cstdint>
+#include <cstring>
 
 #include "h2o_internal.cuh"
 
@@ -33,19 +34,15 @@ namespace {
 constexpr int kTailThreads = 512;
 constexpr int kMaxCluster = 16;
 constexpr uint64_t kNoKey = ~0ull;   // ineligible slot (a real key has pos < 2^31)
-constexpr int kLanes = kTailThreads / kQuarters;   // columns (float4 or float) per round
 constexpr int kDigitBits = 11;                     // radix digit
 constexpr int kBins = 1 << kDigitBits;
 constexpr int kBinsPerThread = kBins / kTailThreads;
 static_assert(kBinsPerThread == 4, "one 16-byte histogram read per thread");
-constexpr int kPre = 8;                            // chunk rows per warp read ahead
-
-__device__ __forceinline__ void add4(float4& a, const float4 b) {
-  a.x += b.x;
-  a.y += b.y;
-  a.z += b.z;
-  a.w += b.w;
-}
+// chunk rows per warp read ahead: 8 in the one-layer kernel; the grouped
+// kernel (many caches per launch) keeps 2 CTAs an SM resident instead, which
+// caps it at 64 registers a thread
+template <int L> constexpr int pre_rows() { return L == 1 ? 8 : 4; }
+template <int L> constexpr int min_blocks() { return L == 1 ? 1 : 2; }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -121,16 +118,25 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t* warp_s
   return before + incl - x;
 }
 
-__global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
+// One launch serves a group of L layers of identical sizes: clusters
+// [l * BH, (l + 1) * BH) take layer l's (b, KV head) caches.
+constexpr int kMaxGroup = 32;
+template <int L>
+struct TailGroup {
+  TailArgs t[L];
+  int BH;
+};
+
+template <int L>
+__global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(const __grid_constant__ TailGroup<L> grp) {
+  constexpr int kPre = pre_rows<L>();
   extern __shared__ __align__(16) unsigned char dyn[];
   uint64_t* keys = reinterpret_cast<uint64_t*>(dyn);                   // [per]
-  float* ns = reinterpret_cast<float*>(dyn + (size_t)p.per * 8);       // [per_s]
+  float* ns = reinterpret_cast<float*>(dyn + (size_t)grp.t[0].per * 8);   // [per_s]
   __shared__ __align__(16) uint32_t hist[3][kBins];   // rank 0's copy is the merged one
   __shared__ __align__(16) uint32_t hloc[kBins];      // this CTA's counts of a pass
   __shared__ uint32_t cnt[kMaxCluster];               // rank 0: selected slots per rank
   __shared__ uint32_t warp_sum[kTailThreads / 32];
-  __shared__ float4 red4[kQuarters - 1][kLanes];      // quarter sums 1..3 of slot columns
-  __shared__ float red1[kQuarters - 1][kLanes];       // ... and of chunk columns
   __shared__ uint64_t sh_prefix, sh_mask;
   __shared__ int64_t sh_kth;
   __shared__ int sh_state;                            // 0 searching, 1 found, 2 too few
@@ -139,7 +145,10 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthr = kTailThreads, nwarps = kTailThreads / 32;
   const uint32_t rank = cluster_rank(), cs = cluster_size();
-  const int64_t bh = blockIdx.x / cs;
+  const int64_t item = blockIdx.x / cs;                 // (layer, b, KV head)
+  const int layer = L == 1 ? 0 : (int)(item / grp.BH);
+  const int64_t bh = item - (int64_t)layer * grp.BH;
+  const TailArgs& p = grp.t[layer];
   const int64_t M = p.M, S = p.S, nv = p.n_valid, need = p.need;
   const int64_t lo = (int64_t)rank * p.per, hi = lo + p.per < M ? lo + p.per : M;
   const int64_t nloc = hi > lo ? hi - lo : 0;
@@ -174,65 +183,23 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
     }
   }
 
-  // ---- 1. scores += partial column sums; keys of the eligible slots; the
-  // chunk rows' initial scores.  A column's partial rows are added in the
-  // kQuarters-run order, here one thread a run; a round covers 4 * kLanes
-  // slots and kLanes chunk columns.
-  const int n_rows = p.n_grp * p.n_rt;
-  const float* base = p.partials + bh * (int64_t)n_rows * p.stride;
+  // ---- 1. scores += summed weights (the accumulator words are read and
+  // cleared for the next chunk); keys of the eligible slots; the chunk rows'
+  // initial scores.  Four slots a thread per round.
+  unsigned long long* acc = p.colacc + bh * p.acc_stride;
   float* sc = p.scores + bh * M;
-  const int32_t* ps = p.pos + bh * M;
+  int32_t* ps = p.pos + bh * M;
   const int64_t lim = p.t0 - p.R;               // eligible: 0 <= pos < t0 - R
-  const int qr = tid / kLanes, ln = tid - qr * kLanes;
-  const int64_t s_end = hi < nv ? hi : nv;      // slots with partial columns
-  const int64_t n_sr = (nloc + 4 * kLanes - 1) / (4 * kLanes);
-  const int64_t n_cr = hi_s > lo_s ? (hi_s - lo_s + kLanes - 1) / kLanes : 0;
-  // With at most kQuarters rows every run of a column's row list holds at most
-  // one row, and the run order is the plain sequential sum: a thread then takes
-  // whole columns (4 slots at a time), with no combine through shared memory.
-  const bool narrow = n_rows <= kQuarters;
-  if (narrow) {
-    for (int64_t s0 = lo + 4 * (int64_t)tid; s0 < hi; s0 += 4 * (int64_t)nthr) {
-      float scv[4] = {0.f, 0.f, 0.f, 0.f};
-      int32_t psv[4] = {-1, -1, -1, -1};
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (s0 + e < hi) {
-          scv[e] = sc[s0 + e];
-          psv[e] = ps[s0 + e];
-        }
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (s0 < s_end)
-        for (int r = 0; r < n_rows; ++r)
-          add4(acc, __ldg(reinterpret_cast<const float4*>(base + s0 + (int64_t)r * p.stride)));
-      const float add[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int64_t s = s0 + e;
-        if (s >= hi) break;
-        float v = scv[e];
-        if (s < nv) {
-          v += add[e];
-          sc[s] = v;
-        }
-        const int32_t q = psv[e];
-        keys[s - lo] = (q >= 0 && q < lim) ? ((uint64_t)ordered_bits(v) << 32) | (uint32_t)q : kNoKey;
-      }
-    }
-    for (int64_t i = lo_s + tid; i < hi_s; i += nthr) {
-      const int rt0 = (int)(i / p.row_tile);      // chunk key i is seen by row tiles rt >= rt0
-      float acc = 0.f;
-      for (int g = 0; g < p.n_grp; ++g)
-        for (int rt = rt0; rt < p.n_rt; ++rt) acc += __ldg(base + (int64_t)(g * p.n_rt + rt) * p.stride + M + i);
-      ns[i - lo_s] = acc;
-    }
-  }
-  const int64_t rounds = narrow ? 0 : (n_sr > n_cr ? n_sr : n_cr);
-  for (int64_t rd = 0; rd < rounds; ++rd) {
-    const int64_t s0 = lo + rd * 4 * kLanes + 4 * ln;
+  const bool vec = (M & 3) == 0;                // rows of scores / positions 16-byte aligned
+  for (int64_t s0 = lo + 4 * (int64_t)tid; s0 < hi; s0 += 4 * (int64_t)nthr) {
     float scv[4] = {0.f, 0.f, 0.f, 0.f};
     int32_t psv[4] = {-1, -1, -1, -1};
-    if (qr == 0) {
+    if (vec && s0 + 4 <= hi) {
+      const float4 f = *reinterpret_cast<const float4*>(sc + s0);
+      const int4 q = *reinterpret_cast<const int4*>(ps + s0);
+      scv[0] = f.x; scv[1] = f.y; scv[2] = f.z; scv[3] = f.w;
+      psv[0] = q.x; psv[1] = q.y; psv[2] = q.z; psv[3] = q.w;
+    } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         if (s0 + e < hi) {
@@ -240,69 +207,44 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
           psv[e] = ps[s0 + e];
         }
     }
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (s0 < s_end) {
-      const float* col = base + s0;
-      const int r_hi = (qr + 1) * n_rows / kQuarters;
-      int r = qr * n_rows / kQuarters;
-      for (; r + 8 <= r_hi; r += 8) {
-        float4 x[8];
+    unsigned long long av[4] = {0ull, 0ull, 0ull, 0ull};
+    if (s0 + 4 <= nv) {                         // acc rows and s0 are multiples of 4 words
+      ulonglong2* a2 = reinterpret_cast<ulonglong2*>(acc + s0);
+      const ulonglong2 x0 = a2[0], x1 = a2[1];
+      av[0] = x0.x; av[1] = x0.y; av[2] = x1.x; av[3] = x1.y;
+      a2[0] = make_ulonglong2(0ull, 0ull);
+      a2[1] = make_ulonglong2(0ull, 0ull);
+    } else {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = __ldg(reinterpret_cast<const float4*>(col + (int64_t)(r + u) * p.stride));
-#pragma unroll
-        for (int u = 0; u < 8; ++u) add4(acc, x[u]);
-      }
-      for (; r < r_hi; ++r) add4(acc, __ldg(reinterpret_cast<const float4*>(col + (int64_t)r * p.stride)));
-    }
-    const int64_t i = lo_s + rd * kLanes + ln;
-    float cacc = 0.f;
-    if (i < hi_s) {
-      const int rt0 = (int)(i / p.row_tile);    // chunk key i is seen by row tiles rt >= rt0
-      const int span = p.n_rt - rt0;
-      const int n = p.n_grp * span;             // rows (group, rt >= rt0), group-major
-      const float* col = base + M + i;
-      const int t_hi = (qr + 1) * n / kQuarters;
-      int t = qr * n / kQuarters;
-      for (; t + 8 <= t_hi; t += 8) {
-        float x[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int g = (t + u) / span, rt = rt0 + (t + u) - g * span;
-          x[u] = __ldg(col + (int64_t)(g * p.n_rt + rt) * p.stride);
+      for (int e = 0; e < 4; ++e)
+        if (s0 + e < nv) {
+          av[e] = acc[s0 + e];
+          acc[s0 + e] = 0ull;
         }
+    }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) cacc += x[u];
-      }
-      for (; t < t_hi; ++t) {
-        const int g = t / span, rt = rt0 + t - g * span;
-        cacc += __ldg(col + (int64_t)(g * p.n_rt + rt) * p.stride);
-      }
+    for (int e = 0; e < 4; ++e) {
+      const int64_t s = s0 + e;
+      if (s >= hi) break;
+      float v = scv[e];
+      if (s < nv) v += colsum_value(av[e], p.fx_inv);
+      scv[e] = v;
+      const int32_t q = psv[e];
+      keys[s - lo] = (q >= 0 && q < lim) ? ((uint64_t)ordered_bits(v) << 32) | (uint32_t)q : kNoKey;
     }
-    if (qr > 0) {
-      red4[qr - 1][ln] = acc;
-      red1[qr - 1][ln] = cacc;
-    }
-    __syncthreads();
-    if (qr == 0) {
-      add4(acc, red4[0][ln]);
-      add4(acc, red4[1][ln]);
-      add4(acc, red4[2][ln]);
-      const float add[4] = {acc.x, acc.y, acc.z, acc.w};
+    if (s0 < nv) {
+      if (vec && s0 + 4 <= hi) {
+        *reinterpret_cast<float4*>(sc + s0) = make_float4(scv[0], scv[1], scv[2], scv[3]);
+      } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int64_t s = s0 + e;
-        if (s >= hi) break;
-        float v = scv[e];
-        if (s < nv) {
-          v += add[e];
-          sc[s] = v;
-        }
-        const int32_t q = psv[e];
-        keys[s - lo] = (q >= 0 && q < lim) ? ((uint64_t)ordered_bits(v) << 32) | (uint32_t)q : kNoKey;
+        for (int e = 0; e < 4; ++e)
+          if (s0 + e < nv) sc[s0 + e] = scv[e];
       }
-      if (i < hi_s) ns[i - lo_s] = ((cacc + red1[0][ln]) + red1[1][ln]) + red1[2][ln];
     }
-    __syncthreads();
+  }
+  for (int64_t i = lo_s + tid; i < hi_s; i += nthr) {
+    ns[i - lo_s] = colsum_value(acc[M + i], p.fx_inv);
+    acc[M + i] = 0ull;
   }
   cluster_sync();   // rank 0's histograms are zero, every CTA has its keys
 
@@ -447,39 +389,35 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const TailArgs p) {
     }
     k_from = kPre;
   }
-  // the rest of the warp's rows, eight at a time: their loads in flight together
+  // the rest of the warp's rows, eight at a time: their loads in flight
+  // together; a row of more than 32 vectors (fp32, d = 128) in two passes
   for (int64_t k0 = k_from; k0 < n_mine; k0 += 32) {
     const int32_t my_slot = k0 + lane < n_mine ? ld_relaxed(fr + lo_s + warp + (k0 + lane) * nwarps) : -1;
     const int kn = n_mine - k0 < 32 ? (int)(n_mine - k0) : 32;
     for (int jb = 0; jb < kn; jb += 8) {
-      uint4 buf[8][2];                                   // a row is at most 64 vectors
+      for (int hv = 0; 32 * hv < vecs2; ++hv) {
+        const int c = lane + 32 * hv;                    // K row then V row
+        uint4 buf[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (jb + u < kn) {
-          const int64_t src = (bh * S + lo_s + warp + (k0 + jb + u) * nwarps) * rv;
-#pragma unroll
-          for (int hv = 0; hv < 2; ++hv) {
-            const int c = lane + 32 * hv;                // K row then V row
-            if (c < vecs2) buf[u][hv] = c < rv ? __ldg(p.k + src + c) : __ldg(p.v + src + c - rv);
+        for (int u = 0; u < 8; ++u) {
+          if (jb + u < kn && c < vecs2) {
+            const int64_t src = (bh * S + lo_s + warp + (k0 + jb + u) * nwarps) * rv;
+            buf[u] = c < rv ? __ldg(p.k + src + c) : __ldg(p.v + src + c - rv);
           }
         }
-      }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (jb + u < kn) {
-          const int64_t i = lo_s + warp + (k0 + jb + u) * nwarps;
-          const int32_t slot = __shfl_sync(0xffffffffu, my_slot, jb + u);
-          if (slot < 0 || slot >= M) {
-            if (lane == 0) atomicOr(p.err, kErrBounds);
-          } else {
-            const int64_t dst = (bh * M + slot) * rv;
-#pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
-              const int c = lane + 32 * hv;
-              if (c < rv) p.kc[dst + c] = buf[u][hv];
-              else if (c < vecs2) p.vc[dst + c - rv] = buf[u][hv];
+        for (int u = 0; u < 8; ++u) {
+          if (jb + u < kn) {
+            const int64_t i = lo_s + warp + (k0 + jb + u) * nwarps;
+            const int32_t slot = __shfl_sync(0xffffffffu, my_slot, jb + u);
+            if (slot < 0 || slot >= M) {
+              if (lane == 0 && hv == 0) atomicOr(p.err, kErrBounds);
+            } else {
+              const int64_t dst = (bh * M + slot) * rv;
+              if (c < rv) p.kc[dst + c] = buf[u];
+              else if (c < vecs2) p.vc[dst + c - rv] = buf[u];
+              if (hv == 0) finish_row(i, slot);
             }
-            finish_row(i, slot);
           }
         }
       }
@@ -499,22 +437,27 @@ constexpr size_t kTailSmemMax = 180 * 1024;   // plus about 41 KB static
 
 }  // namespace
 
-int tail_cluster_size(int64_t M, int64_t S, int BH) {
+int tail_cluster_size(int64_t M, int64_t S, int BH, bool grouped) {
   static_assert(kMaxCluster == 16, "cluster sizes below assume 16");
-  if (cudaFuncSetAttribute(tail_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+  if (cudaFuncSetAttribute(tail_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+      cudaFuncSetAttribute(tail_kernel<kMaxGroup>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
-  // the fewest waves of clusters (all BH at once if possible), then the
-  // largest cluster
+  // the least work per SM along the critical path: waves of clusters times the
+  // share of a cache each CTA takes (1 / cs); on a tie the fewer waves, then the
+  // larger cluster
   int best = 0;
+  double best_cost = 1e300;
   int64_t best_waves = INT64_MAX;
   for (int cs = kMaxCluster; cs >= 1; cs >>= 1) {
     if (cs > 1 && M < 32LL * cs) continue;       // at least 32 slots a CTA
     int per, per_s;
     const size_t smem = tail_smem(M, S, cs, &per, &per_s);
     if (smem > kTailSmemMax) break;               // grows as cs falls: no smaller size fits
-    if (cudaFuncSetAttribute(tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+    const void* kern = grouped ? reinterpret_cast<const void*>(tail_kernel<kMaxGroup>)
+                               : reinterpret_cast<const void*>(tail_kernel<1>);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
       cudaGetLastError();
       break;
     }
@@ -530,13 +473,15 @@ int tail_cluster_size(int64_t M, int64_t S, int BH) {
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, tail_kernel, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
       cudaGetLastError();
       n = 0;
     }
     if (n < 1) continue;
     const int64_t waves = (BH + n - 1) / n;
-    if (waves < best_waves) {
+    const double cost = (double)waves / cs;
+    if (cost < best_cost * (1 - 1e-9) || (cost <= best_cost * (1 + 1e-9) && waves < best_waves)) {
+      best_cost = cost;
       best_waves = waves;
       best = cs;
     }
@@ -544,15 +489,24 @@ int tail_cluster_size(int64_t M, int64_t S, int BH) {
   return best;
 }
 
-cudaError_t launch_tail(const TailArgs& a0, int BH, int cs, bool pdl, cudaStream_t st) {
-  if (cs < 1 || cs > kMaxCluster || (cs & (cs - 1)) != 0) return cudaErrorInvalidValue;
-  TailArgs a = a0;
-  const size_t smem = tail_smem(a.M, a.S, cs, &a.per, &a.per_s);
+namespace {
+
+template <int L>
+cudaError_t launch_tail_t(const TailArgs* a, int n, int BH, int cs, bool pdl, cudaStream_t st) {
+  static_assert(sizeof(TailGroup<L>) <= 32000, "kernel parameter space");
+  TailGroup<L> g;
+  memset(&g, 0, sizeof(g));
+  g.BH = BH;
+  size_t smem = 0;
+  for (int l = 0; l < n; ++l) {
+    g.t[l] = a[l];
+    smem = tail_smem(a[l].M, a[l].S, cs, &g.t[l].per, &g.t[l].per_s);
+  }
   if (smem > kTailSmemMax) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(tail_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(BH * cs));
+  cfg.gridDim = dim3((unsigned)((int64_t)n * BH * cs));
   cfg.blockDim = dim3(kTailThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -565,7 +519,23 @@ cudaError_t launch_tail(const TailArgs& a0, int BH, int cs, bool pdl, cudaStream
   at[1].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, tail_kernel, a);
+  return cudaLaunchKernelEx(&cfg, tail_kernel<L>, g);
+}
+
+}  // namespace
+
+int tail_max_group() { return kMaxGroup; }
+
+cudaError_t launch_tail_group(const TailArgs* a, int n, int BH, int cs, bool pdl, cudaStream_t st) {
+  if (cs < 1 || cs > kMaxCluster || (cs & (cs - 1)) != 0 || n < 1 || n > kMaxGroup)
+    return cudaErrorInvalidValue;
+  for (int l = 1; l < n; ++l)
+    if (a[l].M != a[0].M || a[l].S != a[0].S) return cudaErrorInvalidValue;
+  return n == 1 ? launch_tail_t<1>(a, 1, BH, cs, pdl, st) : launch_tail_t<kMaxGroup>(a, n, BH, cs, pdl, st);
+}
+
+cudaError_t launch_tail(const TailArgs& a, int BH, int cs, bool pdl, cudaStream_t st) {
+  return launch_tail_group(&a, 1, BH, cs, pdl, st);
 }
 
 }  // namespace h2o

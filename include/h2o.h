@@ -36,6 +36,12 @@
  * Pointers: q/k/v/out and every read-back buffer may be device memory or host
  * memory (pinned or pageable); host buffers are staged through library-owned
  * device buffers with stream-ordered copies.  The caller owns all of them.
+ * Host inputs of a step are copied on a stream of the handle's own into one of
+ * two staging sets, so that they overlap the previous step's kernels; the
+ * step's kernels wait for them.  Like device buffers, host buffers may be
+ * reused (inputs) or read (out) once `stream` has passed the step (e.g. after
+ * cudaStreamSynchronize(stream)); with pageable memory the CUDA runtime may
+ * make the copies synchronous.
  * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream); every
  * call only enqueues work on it, except where stated.  A handle is not
  * thread-safe.
@@ -49,9 +55,9 @@
  * not wait for the GPU, so that may be several steps later).  Such a report
  * does not name the step that failed, and every step enqueued since the last
  * point at which the handle was known to be clean (a call that returned after
- * waiting for the GPU: a step with host buffers, a read-back into host memory,
- * or any step while the environment sets H2O_SYNC_CHECK=1) has then run on a
- * cache whose contents are unspecified: destroy the handle.  With
+ * waiting for the GPU: a read-back into host memory, or any step while the
+ * environment sets H2O_SYNC_CHECK=1) has then run on a cache whose contents
+ * are unspecified: destroy the handle.  With
  * H2O_SYNC_CHECK=1 every step waits for its own kernels and reports its own
  * device error.
  */
@@ -107,6 +113,26 @@ int h2o_prefill(h2o_t h, const void* q, const void* k, const void* v, void* out,
  * evictable (valid slots minus the min(R, t0) protected ones).                */
 int h2o_step(h2o_t h, const void* q, const void* k, const void* v, void* out,
              int64_t S, void* stream);
+
+/* One chunk step of S tokens on each of n handles (the layers of a model, or
+ * any caches that take a chunk together): the same result as calling
+ * h2o_step(hs[l], q[l], k[l], v[l], out ? out[l] : NULL, S, stream) for
+ * l = 0 .. n-1.  When the handles have identical sizes and state (M, R, Hq,
+ * Hkv, d, dtype, B, tokens seen) and the chunk takes the one-kernel
+ * tensor-core path (bf16, d = 128), all layers share one attention launch and
+ * one score/select/scatter launch (per group of up to 32 layers), so a partial
+ * last wave of thread blocks is paid once per group and not once per layer
+ * (Table 6 of "Learning how to Forget: Fine-tuning for Long-Context Sparse
+ * Attention": the policy's cost must stay a small share of a training step);
+ * otherwise each layer runs its own launches.  The handles must be distinct;
+ * `out` may be NULL (no outputs) or hold n pointers (each may be NULL).
+ * Profiling (h2o_set_profiling) is read from hs[0]: its timings then cover the
+ * attention and the tail launches of all n layers.
+ * Errors: as h2o_step, for the first handle that fails; H2O_EINVAL for a NULL
+ * or repeated handle.  A failure before any launch leaves every handle as it
+ * was.                                                                        */
+int h2o_step_layers(h2o_t* hs, int n, const void* const* q, const void* const* k,
+                    const void* const* v, void* const* out, int64_t S, void* stream);
 
 /* Copy the state out (each pointer may be NULL to skip it):
  *   slots      [B, Hkv, S_last] int32: the slots the last step (or prefill)
@@ -183,9 +209,10 @@ int h2o_select(const float* scores, const int32_t* positions, int n_heads, int64
  * -- a serving engine that reserves nearly all device memory for its own pool
  * up front, or latency-critical code that cannot afford cudaMalloc's implicit
  * device synchronisation.  It allocates nothing: the caller passes every input
- * and output, and the only scratch (partial column sums and an error word) is
- * a fixed 16 MiB array in the library's static device memory, which every GPU
- * that loads the library holds until the process exits.
+ * and output, and the only scratch (the fixed-point accumulator rows of the
+ * summed weights and an error word) is a fixed 16 MiB array in the library's
+ * static device memory, which every GPU that loads the library holds until the
+ * process exits.
  *
  * Computes steps 1-2 above (attend, summed weights) for one chunk against a
  * caller-owned cache, without touching any handle state:
@@ -194,9 +221,9 @@ int h2o_select(const float* scores, const int32_t* positions, int n_heads, int64
  *   device pointers of `dtype`;
  *   colsum [B, Hkv, M + S] float32 (device): colsum[.., c] for c < M is slot
  *   c's summed weight (0 for c >= n_valid), colsum[.., M + j] chunk key j's.
- * Limit: B * Hq * ceil(S / T) * W <= 4 * 2^20, with W = M + S rounded up to
- * a multiple of 4 and T = 128 (bf16, the tensor-core kernel) or 64 (float32);
- * larger problems return H2O_ESHAPE.
+ * Limit: B * Hkv * W <= 2 * 2^20 (64-bit words), with W = M + S rounded up to
+ * a multiple of 4; larger problems return H2O_ESHAPE.  Each call clears the
+ * words it uses (stream-ordered memsets, no allocation) before its kernels.
  * Set-up: the first call on a device looks up the device address of the
  * scratch array with that device current; make that first call before any
  * stream capture on the device.

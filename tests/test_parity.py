@@ -437,3 +437,114 @@ def test_host_fault_injection(h2o, monkeypatch, kind):
     cache.close()
     s = run_stream(h2o, cfg)
     assert s["chunks"] == 5
+
+
+def _layer_streams(cfg, layers, T):
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    bounds = [(a, b) for a, b in cfg.bounds() if a < T]
+    out = []
+    for layer in layers:
+        Q, K, V = gen_batch(cfg, layer, device="cuda", T=T)
+        out.append(split_chunks(Q, K, V, bounds))
+    return out, bounds
+
+
+@pytest.mark.parametrize("case", ["b4-3layers", "tiny-bf16-35layers", "mixed-fp32"])
+def test_step_layers_matches_single_steps(h2o, monkeypatch, case):
+    """h2o_step_layers gives, bit for bit, what one h2o_step per layer gives: one
+    grid for all layers' attention and one for all tails (b4: three layers of the
+    28-layer workload; 35 small layers: two groups of at most 32), or per-layer
+    launches when the path is not the one-kernel tensor-core one (fp32).  Keys
+    are not split across CTAs here: a grid of one layer may split them where a
+    grid of many layers does not, and a split adds partial outputs in another
+    order (the summed weights are exact integers either way)."""
+    monkeypatch.setenv("H2O_ATTN_SPLIT", "1")
+    if case == "b4-3layers":
+        cfg, n, T = _cfg(4), 3, None
+        T = cfg.P + 3 * cfg.S
+    elif case == "tiny-bf16-35layers":
+        cfg, n = _cfg(0, dtype=torch.bfloat16, d=128, name="tiny-bf16"), 35
+        T = cfg.T
+    else:
+        cfg, n = _cfg(0), 3
+        T = cfg.T
+    streams, bounds = _layer_streams(cfg, range(n), T)
+    mk = lambda: [h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype) for _ in range(n)]  # noqa: E731
+    grouped, single = mk(), mk()
+    for ci in range(len(bounds)):
+        if ci == 0:
+            for l in range(n):
+                grouped[l].prefill(*streams[l][0])
+                single[l].prefill(*streams[l][0])
+            continue
+        outs_g = h2o.step_layers(grouped, [s[ci][0] for s in streams], [s[ci][1] for s in streams],
+                                 [s[ci][2] for s in streams])
+        outs_s = [single[l].step(*streams[l][ci]) for l in range(n)]
+        torch.cuda.synchronize()
+        for l in range(n):
+            assert torch.equal(outs_g[l], outs_s[l]), f"chunk {ci} layer {l}: outputs differ"
+            for x, y in zip(grouped[l].read_state() + grouped[l].read_delta(),
+                            single[l].read_state() + single[l].read_delta()):
+                assert torch.equal(x, y), f"chunk {ci} layer {l}: state differs"
+            assert grouped[l].info()["t0"] == bounds[ci][1]
+    for l in range(n):
+        for x, y in zip(grouped[l].read_kv(), single[l].read_kv()):
+            assert torch.equal(x, y)
+    for c in grouped + single:
+        c.close()
+
+
+def test_step_layers_against_the_oracle(h2o):
+    """Three layers of the 28-layer workload stepped together; sampled (batch,
+    KV head) caches of each layer followed by the oracle along the stream."""
+    cfg = _cfg(4)
+    n, T = 3, cfg.P + 3 * cfg.S
+    streams, bounds = _layer_streams(cfg, [0, 13, 27], T)
+    caches = [h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype) for _ in range(n)]
+    heads = [(1, 2), (3, 7), (0, 5)]
+    G = cfg.G
+    orc = [H2OHeadOracle(cfg.M, cfg.R, G, cfg.d) for _ in range(n)]
+    for ci in range(len(bounds)):
+        pos_before = [o.pos.copy() for o in orc]
+        if ci == 0:
+            outs = [caches[l].prefill(*streams[l][0]) for l in range(n)]
+        else:
+            outs = h2o.step_layers(caches, [s[ci][0] for s in streams], [s[ci][1] for s in streams],
+                                   [s[ci][2] for s in streams])
+        torch.cuda.synchronize()
+        for l in range(n):
+            b, h = heads[l]
+            q, k, v = (to64(x) for x in streams[l][ci])
+            ref = orc[l].step(q[b, h * G:(h + 1) * G], k[b, h], v[b, h])
+            where = f"layer {l} chunk {ci} (b={b}, h={h})"
+            check_outputs(to64(outs[l])[b, h * G:(h + 1) * G], ref, cfg.dtype, where)
+            slots, scores, pos = (x.cpu().numpy() for x in caches[l].read_state())
+            annotate_boundary(orc[l], pos_before[l])
+            if check_evictions(orc[l], slots[b, h], where) == "exact":
+                assert np.array_equal(pos[b, h], orc[l].pos), f"{where}: slot -> position map differs"
+                check_scores(scores[b, h], orc[l].score, orc[l].pos >= 0, where)
+            else:
+                check_tie_state(slots[b, h], pos[b, h], pos_before[l], bounds[ci][0], where)
+                kc, vc = caches[l].read_kv()
+                _sync_head(orc[l], kc, vc, scores, pos, b, h, bounds[ci][1])
+    for c in caches:
+        c.close()
+
+
+def test_step_layers_argument_errors(h2o):
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    cfg = _cfg(0, dtype=torch.bfloat16, d=128)
+    Q, K, V = gen_batch(cfg, 0, device="cuda")
+    ch = split_chunks(Q, K, V, cfg.bounds())
+    a = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    b = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    a.prefill(*ch[0])
+    with pytest.raises(h2o.H2OError) as ei:            # b is not prefilled
+        h2o.step_layers([a, b], [ch[1][0]] * 2, [ch[1][1]] * 2, [ch[1][2]] * 2)
+    assert ei.value.status == -3
+    assert a.info()["t0"] == cfg.P                     # nothing ran
+    with pytest.raises(h2o.H2OError) as ei:            # the same handle twice
+        h2o.step_layers([a, a], [ch[1][0]] * 2, [ch[1][1]] * 2, [ch[1][2]] * 2)
+    assert ei.value.status == -1
+    a.close()
+    b.close()

@@ -66,9 +66,10 @@ def test_noalloc_matches_handle_api_on_two_calls(cuda_ok, dtype, d):
 
 def test_noalloc_rejects_sizes_above_its_scratch(cuda_ok):
     import h2o_kv_cache_b200 as h2o
-    q = torch.zeros(1, 32, 1024, 128, dtype=torch.bfloat16, device="cuda")
-    k = torch.zeros(1, 8, 1024, 128, dtype=torch.bfloat16, device="cuda")
-    kc = torch.zeros(1, 8, 65536, 128, dtype=torch.bfloat16, device="cuda")
+    # 4 * 8 * (65536 + 1024) accumulator words: above the 2 Mi-word array
+    q = torch.zeros(4, 32, 1024, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(4, 8, 1024, 128, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(4, 8, 65536, 128, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(h2o.H2OError) as ei:
         h2o.attend_noalloc(q, k, k, kc, kc, n_valid=65536, M=65536)
     assert ei.value.status == -2 and "fixed maximum" in str(ei.value)
