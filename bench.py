@@ -459,6 +459,10 @@ def measure(args, cfg, world, rank, local, steps, with_e2e):
             host_steps.append(pinned[j])
         h2d = sum(x.numel() * x.element_size() for hs in host_steps[0] for x in hs)
         d2h = sum(o.numel() * o.element_size() for o in houts)
+        # untimed warm-up of the host-buffer path: its staging buffers are
+        # allocated on first use
+        for i in range(2):
+            step_all(houts, host=host_steps[i % len(host_steps)])
         barrier(world)
         for i in range(steps):
             flush.zero_()
@@ -576,6 +580,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the 16k- and 32k-slot workloads measured after the default one")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="run only this many of the workload's layers (a smaller case for profilers)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--clock-poller", type=int, default=None, help=argparse.SUPPRESS)
     args = ap.parse_args()
@@ -585,6 +591,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = workload_module().CONFIGS[args.config]
+    if args.layers is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, layers=max(1, min(args.layers, cfg.layers)))
     if args.impl == "reference":
         run_reference(args, cfg)
     else:
