@@ -21,6 +21,8 @@ from ._lib import (H2O_BF16, H2O_F32, H2O_OK, STATUS_NAMES, lib)
 __all__ = ["H2OCache", "H2OError", "select", "attend_noalloc", "step_layers", "lib"]
 
 _DTYPES = {torch.float32: H2O_F32, torch.bfloat16: H2O_BF16}
+# eviction policies: heavy hitters (h2o) or recency only (lr); see include/h2o.h
+_POLICIES = {"h2o": _lib.H2O_POLICY_H2O, "lr": _lib.H2O_POLICY_LR}
 
 
 class H2OError(RuntimeError):
@@ -49,15 +51,19 @@ class H2OCache:
     """One layer's H2O caches for B sequences (batch fixed at prefill)."""
 
     def __init__(self, M: int, R: int, Hq: int, Hkv: int, d: int, dtype=torch.bfloat16,
-                 device=None):
+                 device=None, policy: str = "h2o"):
         if dtype not in _DTYPES:
             raise ValueError("dtype must be torch.float32 or torch.bfloat16")
+        if policy not in _POLICIES:
+            raise ValueError(f"policy must be one of {sorted(_POLICIES)}")
         self.M, self.R, self.Hq, self.Hkv, self.d, self.dtype = M, R, Hq, Hkv, d, dtype
+        self.policy = policy
         self.device = torch.device(device if device is not None else "cuda", )
         if self.device.index is None:
             self.device = torch.device("cuda", torch.cuda.current_device())
         h = ctypes.c_void_p()
-        _check(lib.h2o_create(M, R, Hq, Hkv, d, _DTYPES[dtype], ctypes.byref(h)))
+        _check(lib.h2o_create_policy(M, R, Hq, Hkv, d, _DTYPES[dtype], _POLICIES[policy],
+                                     ctypes.byref(h)))
         self._h = h
         self.B = None
         self.last_S = None

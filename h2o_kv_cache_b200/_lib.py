@@ -13,6 +13,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libh2o.so")
 
 H2O_OK, H2O_EINVAL, H2O_ESHAPE, H2O_ESTATE, H2O_ENOMEM, H2O_ECUDA, H2O_ETIMEOUT = 0, -1, -2, -3, -4, -5, -6
 H2O_F32, H2O_BF16 = 0, 1
+H2O_POLICY_H2O, H2O_POLICY_LR = 0, 1
 STATUS_NAMES = {0: "H2O_OK", -1: "H2O_EINVAL", -2: "H2O_ESHAPE", -3: "H2O_ESTATE",
                 -4: "H2O_ENOMEM", -5: "H2O_ECUDA", -6: "H2O_ETIMEOUT"}
 
@@ -21,6 +22,7 @@ _i64, _i32, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
 # name -> (restype, argtypes), exactly the declarations of include/h2o.h
 SIGNATURES = {
     "h2o_create": (_i32, [_i64, _i64, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp)]),
+    "h2o_create_policy": (_i32, [_i64, _i64, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp)]),
     "h2o_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i64, _vp]),
     "h2o_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp]),
     "h2o_step_layers": (_i32, [ctypes.POINTER(_vp), _i32, ctypes.POINTER(_vp), ctypes.POINTER(_vp),

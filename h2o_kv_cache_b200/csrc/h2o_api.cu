@@ -35,6 +35,7 @@ int h2o::set_thread_error(int code, const char* msg) {
 struct h2o_ctx {
   int64_t M = 0, R = 0;
   int Hq = 0, Hkv = 0, d = 0, dtype = 0, G = 0, esize = 0;
+  int policy = H2O_POLICY_H2O;
   int B = 0;
   int device = -1;
   int64_t t0 = 0, n_valid = 0, last_S = 0;
@@ -439,6 +440,7 @@ h2o::TailArgs tail_args(const ChunkRun& r) {
   t.need = r.need;
   t.acc_stride = h->acc_stride;
   t.fx_inv = h2o::fx_inv_of(r.fx_shift);
+  t.recency = h->policy == H2O_POLICY_LR ? 1 : 0;
   t.row_vecs = (int)(h->d * elem_size(h->dtype) / 16);
   t.per = t.per_s = 0;
   return t;
@@ -458,7 +460,8 @@ int launch_tail(ChunkRun& r, cudaStream_t st) {
                                  static_cast<float*>(h->newscore.p), BH, r.S, h->M, h->n_valid, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "score reduce launch");
     e = h2o::launch_select(h->scores, h->pos, BH, h->M, h->t0, h->R, r.need, h->n_valid, r.S,
-                           static_cast<int32_t*>(h->freed.p), r.S, h->err, st);
+                           static_cast<int32_t*>(h->freed.p), r.S, h->err, st,
+                           h->policy == H2O_POLICY_LR ? 1 : 0);
     if (e != cudaSuccess) return cuda_fail(h, e, "select launch");
     e = h2o::launch_scatter(r.dk, r.dv, h->kc, h->vc, h->scores, h->pos,
                             static_cast<int32_t*>(h->freed.p), static_cast<float*>(h->newscore.p),
@@ -531,7 +534,7 @@ int run_layers(h2o_ctx** hs, int n, const void* const* q, const void* const* k,
     return h->use_umma && !r.decode && !r.stream && h->tail_cs > 0 && h->device == h0->device &&
            h->B == h0->B && h->Hq == h0->Hq && h->Hkv == h0->Hkv && h->d == h0->d &&
            h->M == h0->M && h->R == h0->R && h->t0 == h0->t0 && h->n_valid == h0->n_valid &&
-           h->tail_cs == h0->tail_cs && r.a.split == runs[0].a.split &&
+           h->tail_cs == h0->tail_cs && h->policy == h0->policy && r.a.split == runs[0].a.split &&
            r.a.inject_timeout == runs[0].a.inject_timeout;
   };
   bool all = true;
@@ -658,7 +661,16 @@ int alloc_state(h2o_ctx* h, int B) {
 extern "C" {
 
 int h2o_create(int64_t M, int64_t R, int Hq, int Hkv, int d, int dtype, h2o_t* out) {
+  return h2o_create_policy(M, R, Hq, Hkv, d, dtype, H2O_POLICY_H2O, out);
+}
+
+int h2o_create_policy(int64_t M, int64_t R, int Hq, int Hkv, int d, int dtype, int policy,
+                      h2o_t* out) {
   if (!out) return fail(nullptr, H2O_EINVAL, "h2o_create: out is NULL");
+  if (policy != H2O_POLICY_H2O && policy != H2O_POLICY_LR) {
+    *out = nullptr;
+    return fail(nullptr, H2O_EINVAL, "h2o_create: unknown policy %d", policy);
+  }
   *out = nullptr;
   if (M < 1 || R < 0 || R >= M)
     return fail(nullptr, H2O_EINVAL, "h2o_create: need M >= 1 and 0 <= R < M (M=%lld R=%lld)",
@@ -679,6 +691,7 @@ int h2o_create(int64_t M, int64_t R, int Hq, int Hkv, int d, int dtype, h2o_t* o
   h->G = Hq / Hkv;
   h->d = d;
   h->dtype = dtype;
+  h->policy = policy;
   h->esize = (int)elem_size(dtype);
   h->use_umma = h2o::attn_umma_supported(dtype, d);
   h->row_tile = h->use_umma ? h2o::kUmmaRowTile : h2o::kSimtRowTile;

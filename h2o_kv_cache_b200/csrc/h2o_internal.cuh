@@ -109,9 +109,11 @@ cudaError_t launch_score_reduce(unsigned long long* colacc, int64_t acc_stride, 
 // freed[bh, 0..S) = ascending evicted slots (need of them), then empty slots
 // n_valid, n_valid + 1, ...  Sets kErrSelect in *err if a head has too few
 // eligible slots.
+// recency = 1 ranks the eligible slots by position alone (the lr policy).
 cudaError_t launch_select(const float* scores, const int32_t* pos, int BH, int64_t M,
                           int64_t t0, int64_t R, int64_t need, int64_t n_valid, int64_t S,
-                          int32_t* freed, int64_t freed_stride, int* err, cudaStream_t st);
+                          int32_t* freed, int64_t freed_stride, int* err, cudaStream_t st,
+                          int recency = 0);
 
 // Chunk token i -> slot freed[bh, i]: K and V rows, pos = t0 + i, score = newscore[bh, i];
 // evicted[bh, i] = the position the slot held before (-1 if it was empty).
@@ -135,6 +137,7 @@ struct TailArgs {
   int* err;
   int64_t M, S, n_valid, t0, R, need, acc_stride;
   float fx_inv;            // 2^-fx_shift
+  int recency;             // 1: rank eligible slots by position alone (lr policy)
   int row_vecs;
   int per, per_s;          // set by launch_tail
 };

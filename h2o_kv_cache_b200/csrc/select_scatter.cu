@@ -48,7 +48,7 @@ __device__ __forceinline__ uint32_t ordered_bits(float x) {
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ pos, int64_t M,
               int64_t t0, int64_t R, int64_t need, int64_t n_valid, int64_t S,
-              int32_t* __restrict__ freed, int64_t freed_stride, int* err) {
+              int32_t* __restrict__ freed, int64_t freed_stride, int* err, int recency) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t warp_tot[kSelThreads / 32];
   __shared__ uint64_t sh_prefix, sh_mask;
@@ -76,7 +76,7 @@ select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ pos,
       if (s < M) {
         const int32_t p = ps[s];
         if (p >= 0 && p < lim) {
-          const uint64_t key = ((uint64_t)ordered_bits(sc[s]) << 32) | (uint32_t)p;
+          const uint64_t key = (recency ? 0ull : (uint64_t)ordered_bits(sc[s]) << 32) | (uint32_t)p;
           if ((key & mask) == prefix) { take = true; digit = (uint32_t)(key >> shift) & 0xFFu; }
         }
       }
@@ -135,7 +135,7 @@ select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ pos,
       if (s < M) {
         const int32_t p = ps[s];
         if (p >= 0 && p < lim) {
-          const uint64_t key = ((uint64_t)ordered_bits(sc[s]) << 32) | (uint32_t)p;
+          const uint64_t key = (recency ? 0ull : (uint64_t)ordered_bits(sc[s]) << 32) | (uint32_t)p;
           sel = (key & mask) <= prefix;
         }
       }
@@ -201,9 +201,9 @@ cudaError_t launch_score_reduce(unsigned long long* colacc, int64_t acc_stride, 
 
 cudaError_t launch_select(const float* scores, const int32_t* pos, int BH, int64_t M, int64_t t0,
                           int64_t R, int64_t need, int64_t n_valid, int64_t S, int32_t* freed,
-                          int64_t freed_stride, int* err, cudaStream_t st) {
+                          int64_t freed_stride, int* err, cudaStream_t st, int recency) {
   select_kernel<<<BH, kSelThreads, 0, st>>>(scores, pos, M, t0, R, need, n_valid, S, freed,
-                                            freed_stride, err);
+                                            freed_stride, err, recency);
   return cudaGetLastError();
 }
 

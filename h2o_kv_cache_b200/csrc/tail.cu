@@ -145,6 +145,12 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthr = kTailThreads, nwarps = kTailThreads / 32;
   const uint32_t rank = cluster_rank(), cs = cluster_size();
+  // a cluster of one CTA needs only the CTA barrier (the cluster barrier's
+  // release would also wait for every global store in flight)
+  auto csync = [&] {
+    if (cs == 1) __syncthreads();
+    else cluster_sync();
+  };
   const int64_t item = blockIdx.x / cs;                 // (layer, b, KV head)
   const int layer = L == 1 ? 0 : (int)(item / grp.BH);
   const int64_t bh = item - (int64_t)layer * grp.BH;
@@ -230,7 +236,9 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
       if (s < nv) v += colsum_value(av[e], p.fx_inv);
       scv[e] = v;
       const int32_t q = psv[e];
-      keys[s - lo] = (q >= 0 && q < lim) ? ((uint64_t)ordered_bits(v) << 32) | (uint32_t)q : kNoKey;
+      keys[s - lo] = (q >= 0 && q < lim)
+                         ? (p.recency ? 0ull : (uint64_t)ordered_bits(v) << 32) | (uint32_t)q
+                         : kNoKey;
     }
     if (s0 < nv) {
       if (vec && s0 + 4 <= hi) {
@@ -246,7 +254,7 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
     ns[i - lo_s] = colsum_value(acc[M + i], p.fx_inv);
     acc[M + i] = 0ull;
   }
-  cluster_sync();   // rank 0's histograms are zero, every CTA has its keys
+  csync();   // rank 0's histograms are zero, every CTA has its keys
 
   // ---- 2. radix select of the need-th smallest key over the cluster,
   // kDigitBits a pass from the top (the last pass takes the 9 bits left)
@@ -285,7 +293,7 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
     // the histogram of the next pass was last read before the previous barrier
     if (rank == 0)
       for (int b = tid; b < kBins; b += nthr) hist[(pass + 1) % 3][b] = 0u;
-    cluster_sync();
+    csync();
     // thread t reads merged bins [kBinsPerThread * t, kBinsPerThread * (t + 1))
     const uint4 h4 = dsmem_ld4(H + (uint32_t)tid * 16u);
     const uint32_t hv[4] = {h4.x, h4.y, h4.z, h4.w};
@@ -326,7 +334,7 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   const uint32_t my_off = block_excl_scan(mine, warp_sum, &cta_sel);
   const uint32_t cnt0 = dsmem_addr(&cnt[0], 0);
   if (tid == 0) dsmem_st(cnt0 + rank * 4u, cta_sel);
-  cluster_sync();
+  csync();
   if (warp == 0) {
     const uint32_t x = lane < (int)cs ? dsmem_ld(cnt0 + (uint32_t)lane * 4u) : 0u;
     const uint32_t off = __reduce_add_sync(0xffffffffu, lane < (int)rank ? x : 0u);
@@ -358,7 +366,7 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
     fr[need + e] = (int32_t)(nv + e);
     ev[need + e] = -1;
   }
-  cluster_sync();   // the freed list is complete; rank 0's shared memory is no longer read
+  csync();   // the freed list is complete; rank 0's shared memory is no longer read
 
   // ---- 4. chunk row i -> slot fr[i]: K and V rows, pos = t0 + i, initial score
   if (!sel_ok) return;
@@ -444,9 +452,27 @@ int tail_cluster_size(int64_t M, int64_t S, int BH, bool grouped) {
     cudaGetLastError();
     return 0;
   }
-  // the least work per SM along the critical path: waves of clusters times the
-  // share of a cache each CTA takes (1 / cs); on a tie the fewer waves, then the
-  // larger cluster
+  // Many caches in one launch (grouped layers): one CTA a cache when there are
+  // at least two waves of them.  The CTAs then need no cluster barriers, and
+  // with two CTAs an SM and more caches than CTA slots the launch streams its
+  // bytes at the HBM rate instead of waiting on barrier latency.
+  if (grouped) {
+    int per, per_s;
+    const size_t smem = tail_smem(M, S, 1, &per, &per_s);
+    int n = 0;
+    if (smem <= kTailSmemMax &&
+        cudaFuncSetAttribute(tail_kernel<kMaxGroup>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, tail_kernel<kMaxGroup>, kTailThreads, smem) == cudaSuccess) {
+      int dev = 0, sms = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+          n > 0 && BH >= 2 * n * sms)
+        return 1;
+    }
+    cudaGetLastError();
+  }
+  // otherwise the least work per SM along the critical path: waves of clusters
+  // times the share of a cache each CTA takes (1 / cs); on a tie the fewer
+  // waves, then the larger cluster
   int best = 0;
   double best_cost = 1e300;
   int64_t best_waves = INT64_MAX;

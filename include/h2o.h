@@ -85,6 +85,19 @@ typedef enum {
 
 typedef enum { H2O_F32 = 0, H2O_BF16 = 1 } h2o_dtype;
 
+/* Eviction policy of a handle.
+ *   H2O_POLICY_H2O  the heavy-hitter policy described at the top: evict the
+ *                   `need` eligible slots with the smallest (score, pos).
+ *   H2O_POLICY_LR   recency only: evict the `need` eligible slots holding the
+ *                   oldest tokens (smallest pos), so the cache holds the most
+ *                   recent tokens.  The page "Learning how to Forget: Fine-
+ *                   tuning for Long-Context Sparse Attention" names an `lr`
+ *                   policy beside `h2o` (Tables 1 and 6) without defining
+ *                   it; this is the plainest reading of the name.  Attention,
+ *                   summed weights and scores are computed as for H2O (the
+ *                   scores are kept but do not decide evictions).            */
+typedef enum { H2O_POLICY_H2O = 0, H2O_POLICY_LR = 1 } h2o_policy;
+
 /* Create a handle for one layer's caches.
  *   M    cache capacity (slots) per (batch, KV head), M >= 1
  *   R    protected recent window in tokens, 0 <= R < M
@@ -95,6 +108,12 @@ typedef enum { H2O_F32 = 0, H2O_BF16 = 1 } h2o_dtype;
  * then).  The scale is fixed at 1/sqrt(d); natural-base softmax.
  * Returns H2O_OK and *out, or H2O_EINVAL.                                     */
 int h2o_create(int64_t M, int64_t R, int Hq, int Hkv, int d, int dtype, h2o_t* out);
+
+/* h2o_create with an eviction policy (h2o_policy); h2o_create is
+ * h2o_create_policy(..., H2O_POLICY_H2O, out).  H2O_EINVAL for an unknown
+ * policy.                                                                     */
+int h2o_create_policy(int64_t M, int64_t R, int Hq, int Hkv, int d, int dtype, int policy,
+                      h2o_t* out);
 
 /* Prefill: the first chunk, P tokens (1 <= P <= M), causal attention among
  * themselves with an empty cache.  Token t goes to slot t with score = its

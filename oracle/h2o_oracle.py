@@ -51,6 +51,7 @@ import numpy as np
 __all__ = [
     "attend_group",
     "select_evictions",
+    "select_oldest",
     "H2OHeadOracle",
     "H2OOracle",
     "OracleShapeError",
@@ -125,10 +126,31 @@ def select_evictions(score, pos, t0, R, need):
     return sorted(ranked[:need])
 
 
-class H2OHeadOracle:
-    """State and step of one (batch, KV head) cache; eviction is per KV head."""
+def select_oldest(pos, t0, R, need):
+    """Slots to evict under the recency-only policy: the `need` eligible slots
+    holding the oldest tokens (smallest pos), ascending by slot.
 
-    def __init__(self, M, R, G, d):
+    The page names an `lr` policy beside `h2o` (Tables 1 and 6) without
+    defining it; the reading taken is the plainest one for its name: keep the
+    most recent tokens.  Eligibility is the same as for H2O (valid, and older
+    than the protected recent window).  Written as a plain Python sort on pos.
+    """
+    pos = np.asarray(pos)
+    eligible = [s for s in range(pos.shape[0]) if pos[s] >= 0 and pos[s] < t0 - R]
+    if need > len(eligible):
+        raise OracleShapeError(f"need {need} evictions but only {len(eligible)} eligible slots")
+    ranked = sorted(eligible, key=lambda s: int(pos[s]))
+    return sorted(ranked[:need])
+
+
+class H2OHeadOracle:
+    """State and step of one (batch, KV head) cache; eviction is per KV head.
+    policy "h2o" (heavy hitters, the default) or "lr" (recency only)."""
+
+    def __init__(self, M, R, G, d, policy="h2o"):
+        if policy not in ("h2o", "lr"):
+            raise ValueError(f"unknown policy {policy!r}")
+        self.policy = policy
         self.M, self.R, self.G, self.d = int(M), int(R), int(G), int(d)
         self.K = np.zeros((self.M, self.d), dtype=np.float64)
         self.V = np.zeros((self.M, self.d), dtype=np.float64)
@@ -169,7 +191,10 @@ class H2OHeadOracle:
             raise OracleShapeError(f"chunk of {S} tokens exceeds cache capacity {self.M}")
         self.last_eligible = (self.pos >= 0) & (self.pos < t0 - self.R)
         self.last_need = need
-        evicted = select_evictions(self.score, self.pos, t0, self.R, need)
+        if self.policy == "h2o":
+            evicted = select_evictions(self.score, self.pos, t0, self.R, need)
+        else:
+            evicted = select_oldest(self.pos, t0, self.R, need)
         freed = sorted(evicted + empties[: S - need])
         # scatter: ascending freed slot <-> ascending new position
         for i, s in enumerate(freed):
@@ -186,9 +211,10 @@ class H2OOracle:
     """All (batch, KV head) caches of one layer; layouts as the library's:
     q, out [B, Hq, S, d]; k, v [B, Hkv, S, d]; query head g uses KV head g // G."""
 
-    def __init__(self, M, R, Hq, Hkv, d, heads=None):
+    def __init__(self, M, R, Hq, Hkv, d, heads=None, policy="h2o"):
         if Hq % Hkv:
             raise ValueError("Hq must be a multiple of Hkv")
+        self.policy = policy
         self.M, self.R, self.Hq, self.Hkv, self.d = int(M), int(R), int(Hq), int(Hkv), int(d)
         self.G = self.Hq // self.Hkv
         self.B = None
@@ -207,7 +233,8 @@ class H2OOracle:
         if P > self.M:
             raise OracleShapeError(f"prefill of {P} tokens exceeds cache capacity {self.M}")
         self.B = B
-        self.heads = {bh: H2OHeadOracle(self.M, self.R, self.G, self.d) for bh in self._head_list()}
+        self.heads = {bh: H2OHeadOracle(self.M, self.R, self.G, self.d, self.policy)
+                      for bh in self._head_list()}
         self.t0 = 0
         return self.step(q, k, v)
 

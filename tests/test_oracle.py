@@ -335,3 +335,63 @@ def test_pins_catch_planted_slips(monkeypatch, target, mutant):
         except (AssertionError, OracleShapeError):
             caught += 1
     assert caught >= 1, f"no pin caught the planted slip in {target}"
+
+
+# --------------------------------------------------------------------------------------
+# The recency-only policy (lr): closed form and windowed attention from a library routine
+# --------------------------------------------------------------------------------------
+def _lr_stream(select=None, seed=7, Hq=4, Hkv=2, d=8, M=24, R=5, P=16, S=6, T=16 + 6 * 8 + 3, B=2):
+    rng = np.random.default_rng(seed)
+    q, k, v = _rand_stream(rng, Hq, Hkv, T, d, B=B)
+    orc = H2OOracle(M, R, Hq, Hkv, d, policy="lr")
+    bounds = [(0, P)] + [(t, min(T, t + S)) for t in range(P, T, S)]
+    outs, cached = [], []
+    for i, (a, b) in enumerate(bounds):
+        x = (q[:, :, a:b], k[:, :, a:b], v[:, :, a:b])
+        outs.append(orc.prefill(*x) if i == 0 else orc.step(*x))
+        cached.append({bh: sorted(int(p) for p in st.pos if p >= 0) for bh, st in orc.heads.items()})
+    return q, k, v, orc, bounds, np.concatenate(outs, axis=2), cached
+
+
+def check_lr_holds_the_most_recent_tokens():
+    M = 24
+    *_, bounds, _, cached = _lr_stream(M=M)
+    for (a, b), c in zip(bounds, cached):
+        for heads in c.values():
+            assert heads == list(range(max(0, b - M), b)), (b, heads)
+
+
+def test_lr_holds_the_most_recent_tokens():
+    # closed form: with M - R >= S the oldest tokens are always evictable, so after
+    # every chunk the cache holds exactly the last M positions
+    check_lr_holds_the_most_recent_tokens()
+
+
+def test_lr_outputs_equal_chunked_window_attention():
+    # the query at t0 + i of a chunk starting at t0 sees positions
+    # [max(0, t0 - M), t0 + i]: library SDPA with that explicit mask, float64
+    M, Hq, Hkv, d = 24, 4, 2, 8
+    q, k, v, orc, bounds, got, _ = _lr_stream(M=M, Hq=Hq, Hkv=Hkv, d=d)
+    T = q.shape[2]
+    allow = torch.zeros(T, T, dtype=torch.bool)
+    for a, b in bounds:
+        for t in range(a, b):
+            allow[t, max(0, a - M):t + 1] = True
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=allow,
+                                                           enable_gqa=True).numpy()
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # the summed weights still carry S * G of mass per KV head and chunk
+    for st in orc.heads.values():
+        S = bounds[-1][1] - bounds[-1][0]
+        assert abs(st.last_c_slots.sum() + st.last_c_new.sum() - S * (Hq // Hkv)) < 1e-9
+
+
+def test_lr_pin_catches_a_newest_first_slip(monkeypatch):
+    # a plausible slip -- evicting the newest eligible tokens -- fails the closed form
+    def newest(pos, t0, R, need):
+        elig = [s for s in range(len(pos)) if 0 <= pos[s] < t0 - R]
+        return sorted(sorted(elig, key=lambda s: -int(pos[s]))[:need])
+    monkeypatch.setattr(ho, "select_oldest", newest)
+    with pytest.raises(AssertionError):
+        check_lr_holds_the_most_recent_tokens()

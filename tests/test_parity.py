@@ -38,7 +38,8 @@ def _sync_head(st, kc, vc, scores, pos, b, h, t0):
     st.load_state(to64(kc[b, h]), to64(vc[b, h]), scores[b, h], pos[b, h], t0)
 
 
-def run_stream(h2o, cfg, heads=None, layer=0, T=None, oracle_chunks=None, kv_check=True):
+def run_stream(h2o, cfg, heads=None, layer=0, T=None, oracle_chunks=None, kv_check=True,
+               policy="h2o"):
     """Returns a summary dict.  oracle_chunks=None: the oracle follows the whole
     stream; otherwise only the listed chunk indices are checked, each after
     loading the GPU's pre-step state into the oracle."""
@@ -48,11 +49,11 @@ def run_stream(h2o, cfg, heads=None, layer=0, T=None, oracle_chunks=None, kv_che
     bounds = [(a, b) for a, b in cfg.bounds() if a < T]
     bounds[-1] = (bounds[-1][0], min(bounds[-1][1], T))
     chunks = split_chunks(Q, K, V, bounds)
-    cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    cache = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype, policy=policy)
     G = cfg.G
     if heads is None:
         heads = [(b, h) for b in range(cfg.B) for h in range(cfg.Hkv)]
-    orc = {bh: H2OHeadOracle(cfg.M, cfg.R, G, cfg.d) for bh in heads}
+    orc = {bh: H2OHeadOracle(cfg.M, cfg.R, G, cfg.d, policy) for bh in heads}
     Kn, Vn = to64(K), to64(V)
     summary = {"chunks": 0, "ties": 0, "max_abs": 0.0, "rel_norm": 0.0, "score_rel": 0.0}
     for ci, (q, k, v) in enumerate(chunks):
@@ -84,6 +85,8 @@ def run_stream(h2o, cfg, heads=None, layer=0, T=None, oracle_chunks=None, kv_che
             summary["max_abs"] = max(summary["max_abs"], r["max_abs"])
             summary["rel_norm"] = max(summary["rel_norm"], r["rel_norm"])
             annotate_boundary(st, pos_before[(b, h)])
+            if policy == "lr":   # positions are unique: the evicted set is fixed, no ties
+                assert np.array_equal(slots[b, h], st.last_freed), f"{where}: filled slots differ"
             status = check_evictions(st, slots[b, h], where)
             if status == "exact":
                 assert np.array_equal(pos[b, h], st.pos), f"{where}: slot -> position map differs"
@@ -548,3 +551,21 @@ def test_step_layers_argument_errors(h2o):
     assert ei.value.status == -1
     a.close()
     b.close()
+
+
+@pytest.mark.parametrize("case", ["tiny-fp32", "ragged-bf16", "m2k-s1k"])
+def test_lr_policy(h2o, case):
+    """The recency-only policy: the same attention, summed weights and scores as
+    H2O, evictions by position; every step matches the oracle exactly and the
+    cache holds the last M tokens."""
+    cfgs = {
+        "tiny-fp32": _cfg(0, name="lr-tiny"),
+        "ragged-bf16": _cfg(0, name="lr-ragged", B=2, Hq=6, Hkv=2, d=128, M=300, R=17,
+                            T=100 + 37 * 7 + 11, P=100, S=37, dtype=torch.bfloat16, planted=0.02),
+        "m2k-s1k": _cfg(1, name="lr-m2k"),
+    }
+    cfg = cfgs[case]
+    T = cfg.P + 4 * cfg.S if case == "m2k-s1k" else None
+    heads = [(0, 2), (0, 5)] if case == "m2k-s1k" else None
+    s = run_stream(h2o, cfg, heads=heads, T=T, policy="lr")
+    assert s["ties"] == 0
