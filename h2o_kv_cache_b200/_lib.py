@@ -9,7 +9,10 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libh2o.so")
+# H2O_LIBRARY names another build of the same library to load instead (the
+# stamps build of stamps.py); unset, the in-tree libh2o.so
+LIB_PATH = os.environ.get("H2O_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                         "libh2o.so")
 
 H2O_OK, H2O_EINVAL, H2O_ESHAPE, H2O_ESTATE, H2O_ENOMEM, H2O_ECUDA, H2O_ETIMEOUT = 0, -1, -2, -3, -4, -5, -6
 H2O_F32, H2O_BF16 = 0, 1
@@ -51,6 +54,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
+    if hasattr(lib, "h2o_stamps_read"):   # only the stamps build of stamps.py exports it
+        lib.h2o_stamps_read.restype = _i32
+        lib.h2o_stamps_read.argtypes = [_vp]
     return lib
 
 

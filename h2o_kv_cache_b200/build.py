@@ -38,11 +38,11 @@ def _deps():
     return max((os.path.getmtime(h) for h in hdrs), default=0.0)
 
 
-def _compile(nvcc, src, verbose):
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(nvcc, src, verbose, build_dir=BUILD, extra=()):
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     if os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), _deps()):
         return obj
-    cmd = [nvcc] + NVCC_FLAGS + ["-c", src, "-o", obj]
+    cmd = [nvcc] + NVCC_FLAGS + list(extra) + ["-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
@@ -54,23 +54,29 @@ def _compile(nvcc, src, verbose):
     return obj
 
 
-def build(verbose: bool = False) -> str:
-    """Compile and link; returns the path of libh2o.so."""
+def build(verbose: bool = False, stamps: bool = False) -> str:
+    """Compile and link; returns the path of libh2o.so.  stamps=True builds the
+    instrumented variant instead (-DH2O_STAMPS: the tensor-core attention kernel
+    records pipeline stamps, see stamps.py) as libh2o_stamps.so, from objects of
+    its own."""
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    build_dir = BUILD + "_stamps" if stamps else BUILD
+    lib = os.path.join(PKG, "libh2o_stamps.so") if stamps else LIB
+    extra = ["-DH2O_STAMPS"] if stamps else []
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(nvcc, s, verbose), srcs))
+        objs = list(ex.map(lambda s: _compile(nvcc, s, verbose, build_dir, extra), srcs))
     newest = max(os.path.getmtime(o) for o in objs)
-    if not os.path.exists(LIB) or os.path.getmtime(LIB) < newest:
-        tmp = LIB + ".tmp"
+    if not os.path.exists(lib) or os.path.getmtime(lib) < newest:
+        tmp = lib + ".tmp"
         cmd = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv))
+    print(build(verbose="--verbose" in sys.argv, stamps="--stamps" in sys.argv))

@@ -49,6 +49,41 @@
 
 #include "attn_common.cuh"
 
+// Pipeline stamps: with -DH2O_STAMPS (a separate build, see
+// h2o_kv_cache_b200/stamps.py) the CTAs of the first wave record clock64() at
+// the hand-offs of their first unit -- per 256-key pair of sweep 1 and per
+// 128-key tile of sweep 2 -- into a file-scope array that h2o_stamps_read()
+// copies out.  The default build compiles every stamp to nothing.
+#ifdef H2O_STAMPS
+namespace h2o_stamps {
+constexpr int kCtas = 148, kSlots = 1200;
+}
+__device__ unsigned long long g_h2o_stamps[h2o_stamps::kCtas * h2o_stamps::kSlots];
+#define H2O_STAMP(i)                                                                     \
+  do {                                                                                   \
+    if (blockIdx.x < h2o_stamps::kCtas && (i) < h2o_stamps::kSlots)                       \
+      g_h2o_stamps[blockIdx.x * h2o_stamps::kSlots + (i)] = clock64();                  \
+  } while (0)
+extern "C" int h2o_stamps_read(unsigned long long* host) {
+  return cudaMemcpyFromSymbol(host, g_h2o_stamps, sizeof(g_h2o_stamps)) == cudaSuccess ? 0 : -1;
+}
+#else
+#define H2O_STAMP(i) \
+  do {               \
+  } while (0)
+#endif
+// stamp slots: [0, 64) producer issues pair u's K tile; [64, 128) MMA warp sees it;
+// [128, 256) MMA warp sees head w's S buffer free (128 + 64 w + u); [256, 320) pair
+// u's MMAs issued; [320, 448) softmax sees head w's S of pair u; [448, 512) softmax
+// ends pair u; sweep 2 tile j: [512, 608) MMA warp starts S^T(j); [608, 704) its
+// waits done; [704, 800) O^T(j)'s waits done; [800, 896) softmax sees S^T(j);
+// [896, 992) sees P^T free; [992, 1088) has stored P^T(j); 1100 start, 1101 end of
+// sweep 1, 1102 end of sweep 2.
+enum : int { kStIssueK = 0, kStKFull = 64, kStSEmpty = 128, kStPairIssued = 256, kStSFull = 320,
+             kStPairEnd = 448, kStStStart = 512, kStStReady = 608, kStOtReady = 704,
+             kStStFull = 800, kStPEmpty = 896, kStPFull = 992, kStStart = 1100,
+             kStSweep1End = 1101, kStSweep2End = 1102 };
+
 namespace h2o {
 namespace {
 
@@ -195,6 +230,7 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
   const uint32_t tmem = *tmem_slot;
   // the cache and the accumulator row may still be in use by the previous kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (threadIdx.x == 0) H2O_STAMP(kStStart);
 
   // local tile t (128 keys), i.e. the unit's tile t_lo + t: tensor map and row offset
   auto tile_src = [&](int t, bool v, const CUtensorMap*& m, int& y) {
@@ -234,6 +270,7 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
         ok = mbar_wait(bar(B_R1_EMPTY + s), ((uint32_t)(u >> 1) & 1u) ^ 1u, abort_flag, err,
                        kWaitLimitNs, kErrTimeout);
         if (!ok) break;
+        if (u < 64) H2O_STAMP(kStIssueK + u);
         const uint32_t dst = base + kOffR + (uint32_t)s * kSlot1;
         mbar_arrive_expect_tx(bar(B_R1_FULL + s), kSlot1);
         for (int half = 0; half < 2; ++half) {
@@ -294,11 +331,13 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
         const int s = u & 1;
         ok = mbar_wait(bar(B_R1_FULL + s), (uint32_t)(u >> 1) & 1u, abort_flag, err, kWaitLimitNs,
                        kErrTimeout);
+        if (u < 64) H2O_STAMP(kStKFull + u);
         const uint32_t k_addr = base + kOffR + (uint32_t)s * kSlot1;
         for (int w = 0; ok && w < 2; ++w) {
           ok = mbar_wait(bar(B_S_EMPTY + w), ((uint32_t)u & 1u) ^ 1u, abort_flag, err, kWaitLimitNs,
                          kErrTimeout);
           if (!ok) break;
+          if (u < 64) H2O_STAMP(kStSEmpty + 64 * w + u);
           tc_fence_after();
           const uint32_t a0 = desc_lo(q_addr + (uint32_t)w * kAtom, 16), b0 = desc_lo(k_addr, 16);
 #pragma unroll
@@ -308,9 +347,11 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
           umma_commit(bar(B_S_FULL + w));
         }
         if (ok) umma_commit(bar(B_R1_EMPTY + s));
+        if (u < 64) H2O_STAMP(kStPairIssued + u);
       }
       // ---- sweep 2: S^T(0), S^T(1), O^T(0), S^T(2), O^T(1), ...
       auto issue_st = [&](int j) -> bool {
+        if (j < 96) H2O_STAMP(kStStStart + j);
         // TMEM columns 0-255: head A's last sweep-1 S, then S^T(j - 1), must have been read
         bool w_ok = (j == 0)
             ? mbar_wait(bar(B_S_EMPTY + 0), ((uint32_t)n1 & 1u) ^ 1u, abort_flag, err, kWaitLimitNs, kErrTimeout)
@@ -320,6 +361,7 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
           w_ok = mbar_wait(bar(B_R2_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, err,
                            kWaitLimitNs, kErrTimeout);
         if (!w_ok) return false;
+        if (j < 96) H2O_STAMP(kStStReady + j);
         tc_fence_after();
         const uint32_t a0 = desc_lo(base + kOffR + (uint32_t)slot * kTile, 16), b0 = desc_lo(q_addr, 16);
 #pragma unroll
@@ -341,6 +383,7 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
           w_ok = mbar_wait(bar(B_R2_FULL + slot), (uint32_t)(pos / NS2) & 1u, abort_flag, err,
                            kWaitLimitNs, kErrTimeout);
         if (!w_ok) return false;
+        if (j < 96) H2O_STAMP(kStOtReady + j);
         tc_fence_after();
         const uint32_t a0 = desc_lo(base + kOffR + (uint32_t)slot * kTile, kAtom), b0 = desc_lo(p_addr, kAtom);
 #pragma unroll
@@ -401,6 +444,7 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
       for (int hw = 0; hw < 2; ++hw) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + hw), (uint32_t)u & 1u, abort_flag, err,
                                                kWaitLimitNs, kErrTimeout));
+        if (threadIdx.x == 64 && u < 64) H2O_STAMP(kStSFull + 64 * hw + u);
         if (!ok) break;
         tc_fence_after();
         const uint32_t s_tmem = lane_base + (uint32_t)hw * 256u + (uint32_t)w * 128u;
@@ -418,6 +462,7 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
         }
       }
       __syncwarp();
+      if (threadIdx.x == 64 && u < 64) H2O_STAMP(kStPairEnd + u);
     }
     // warpgroup w finishes head w's rows: it takes the other warpgroup's
     // (max, sum) of them from shared memory.  Every warp passes both barriers
@@ -472,6 +517,7 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
         for (int q = 0; q < kc; ++q) mbar_arrive_remote(cluster_map(bar(B_X_READ), (uint32_t)q));
     }
     named_bar_sync(1 + w, 128);
+    if (threadIdx.x == 64) H2O_STAMP(kStSweep1End);
 
     // ----- sweep 2: thread = key (lane r of S^T), the 128 query columns of head w;
     // each warpgroup adds its head's column sum of the key to the accumulator row
@@ -484,6 +530,7 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ST_FULL), (uint32_t)j & 1u, abort_flag, err,
                                              kWaitLimitNs, kErrTimeout));
       if (!ok) break;
+      if (threadIdx.x == 64 && j < 96) H2O_STAMP(kStStFull + j);
       tc_fence_after();
       const int jg = t_lo + j;
       const bool cache = jg < nct;
@@ -524,14 +571,17 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_P_EMPTY), ((uint32_t)j & 1u) ^ 1u, abort_flag,
                                              err, kWaitLimitNs, kErrTimeout));
       if (!ok) break;
+      if (threadIdx.x == 64 && j < 96) H2O_STAMP(kStPEmpty + j);
       store_p_half(p_row, r, pk);
       store_p_half(p_row + kAtom, r, pk2);
       fence_async_smem();
       mbar_arrive(bar(B_P_FULL));
+      if (threadIdx.x == 64 && j < 96) H2O_STAMP(kStPFull + j);
       // without a head B every probability of warpgroup 1 is 0
       if (key_ok && head_ok) colsum_add(acc + (cache ? key : M + key), cs_total(cs4), p.fx_scale);
     }
 
+    if (threadIdx.x == 64) H2O_STAMP(kStSweep2End);
     // ----- epilogue: O^T (lane = d, columns = queries) -> out rows via shared memory
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), 0, abort_flag, err,
                                                    kWaitLimitNs, kErrTimeout));

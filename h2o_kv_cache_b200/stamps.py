@@ -1,0 +1,132 @@
+"""Pipeline stamps of the tensor-core attention kernel (a developer tool).
+
+    python -m h2o_kv_cache_b200.stamps [--config 4] [--layers 2] [--steps 3]
+
+Builds the instrumented library (build.py --stamps: the attention kernel compiled
+with -DH2O_STAMPS records clock64() at its hand-offs), runs a few chunk steps of
+a workload on it in a child process, and prints, per 256-key pair of sweep 1 and
+per 128-key tile of sweep 2, the medians over the first wave's CTAs of how long
+each role waited on the others and how long the softmax took.  Needs a B200.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import subprocess
+import sys
+import tempfile
+
+import numpy as np
+
+KCTAS, KSLOTS = 148, 1200
+# slot bases, as in csrc/attn_umma.cu
+ISSUE_K, K_FULL, S_EMPTY, PAIR_ISSUED, S_FULL, PAIR_END = 0, 64, 128, 256, 320, 448
+ST_START, ST_READY, OT_READY, ST_FULL, P_EMPTY, P_FULL = 512, 608, 704, 800, 896, 992
+START, SWEEP1_END, SWEEP2_END = 1100, 1101, 1102
+
+
+def _child(cfg_id, layers, steps, out_path):
+    import ctypes
+    import dataclasses
+
+    import torch
+
+    import h2o_kv_cache_b200 as h2o
+    from h2o_kv_cache_b200.workload import CONFIGS, gen_batch, split_chunks
+    cfg = dataclasses.replace(CONFIGS[cfg_id], layers=layers)
+    T = cfg.P + (steps + 1) * cfg.S
+    bounds = [(a, b) for a, b in cfg.bounds() if a < T]
+    caches, chunks = [], []
+    for layer in range(cfg.layers):
+        Q, K, V = gen_batch(cfg, layer, device="cuda", T=T)
+        ch = split_chunks(Q, K, V, bounds)
+        c = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+        c.prefill(*ch[0])
+        caches.append(c)
+        chunks.append(ch)
+    for i in range(1, min(steps + 1, len(bounds))):
+        if len(caches) > 1:
+            h2o.step_layers(caches, [c[i][0] for c in chunks], [c[i][1] for c in chunks],
+                            [c[i][2] for c in chunks])
+        else:
+            caches[0].step(*chunks[0][i])
+    torch.cuda.synchronize()
+    buf = (ctypes.c_ulonglong * (KCTAS * KSLOTS))()
+    if h2o.lib.h2o_stamps_read(buf) != 0:
+        raise RuntimeError("h2o_stamps_read failed")
+    np.save(out_path, np.frombuffer(buf, dtype=np.uint64).reshape(KCTAS, KSLOTS).astype(np.int64))
+
+
+def summarize(st):
+    """Median (over CTAs) of per-CTA mean waits, in SM clock cycles."""
+    out = {}
+    s1 = []
+    for c in range(st.shape[0]):
+        end = st[c, PAIR_END:PAIR_END + 64]
+        n = int((end > 0).sum())
+        if n < 4:
+            continue
+        u = np.arange(2, n - 1)
+        s1.append([(end[u] - end[u - 1]).mean(),
+                   (st[c, S_FULL + u] - end[u - 1]).mean(),
+                   (st[c, S_FULL + 64 + u] - st[c, S_FULL + u]).mean(),
+                   (end[u] - st[c, S_FULL + 64 + u]).mean(),
+                   (st[c, K_FULL + u] - st[c, PAIR_ISSUED + u - 1]).mean(),
+                   (st[c, S_EMPTY + u] - st[c, K_FULL + u]).mean()])
+    names1 = ["period per 256-key pair", "softmax waits for head A's S", "head A (softmax, then waits for B's S)",
+              "head B softmax", "MMA warp waits for the K tile", "MMA warp waits for head A's S buffer"]
+    if s1:
+        out["sweep 1"] = dict(zip(names1, np.median(np.array(s1), axis=0)))
+    s2 = []
+    for c in range(st.shape[0]):
+        pf = st[c, P_FULL:P_FULL + 96]
+        n = int((pf > 0).sum())
+        if n < 6:
+            continue
+        j = np.arange(2, n - 1)
+        s2.append([(pf[j] - pf[j - 1]).mean(),
+                   (st[c, ST_FULL + j] - pf[j - 1]).mean(),
+                   (st[c, P_EMPTY + j] - st[c, ST_FULL + j]).mean(),
+                   (pf[j] - st[c, P_EMPTY + j]).mean(),
+                   (st[c, ST_READY + j] - st[c, ST_START + j]).mean(),
+                   (st[c, OT_READY + j - 1] - st[c, ST_READY + j]).mean()])
+    names2 = ["period per 128-key tile", "softmax waits for S^T", "exponentials (and wait for the P^T buffer)",
+              "P^T stores", "MMA warp waits before S^T", "MMA warp waits before O^T"]
+    if s2:
+        out["sweep 2"] = dict(zip(names2, np.median(np.array(s2), axis=0)))
+    ok = st[:, START] > 0
+    out["unit"] = {"start to end of sweep 1": float(np.median(st[ok, SWEEP1_END] - st[ok, START])),
+                   "start to end of sweep 2": float(np.median(st[ok, SWEEP2_END] - st[ok, START]))}
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--layers", type=int, default=2)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--child", default=None, help=argparse.SUPPRESS)
+    args = ap.parse_args()
+    if args.child:
+        _child(args.config, args.layers, args.steps, args.child)
+        return
+    here = os.path.dirname(os.path.abspath(__file__))
+    sys.path.insert(0, here)
+    import build as B
+    lib = B.build(stamps=True)
+    out = os.path.join(tempfile.mkdtemp(), "stamps.npy")
+    env = dict(os.environ, H2O_LIBRARY=lib)
+    subprocess.run([sys.executable, "-m", "h2o_kv_cache_b200.stamps", "--config", str(args.config),
+                    "--layers", str(args.layers), "--steps", str(args.steps), "--child", out],
+                   check=True, env=env, cwd=os.path.dirname(here))
+    res = summarize(np.load(out))
+    print(f"workload config {args.config}, {args.layers} layer(s), last of {args.steps} steps; "
+          "medians over the first wave's CTAs, SM clock cycles")
+    for part, vals in res.items():
+        print(part)
+        for k, v in vals.items():
+            print(f"  {k:48s} {v:10.0f}")
+
+
+if __name__ == "__main__":
+    main()
