@@ -54,9 +54,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
-    if hasattr(lib, "h2o_stamps_read"):   # only the stamps build of stamps.py exports it
-        lib.h2o_stamps_read.restype = _i32
-        lib.h2o_stamps_read.argtypes = [_vp]
+    for extra in ("h2o_stamps_read", "h2o_tail_stamps_read"):   # the stamps build only (stamps.py)
+        if hasattr(lib, extra):
+            getattr(lib, extra).restype = _i32
+            getattr(lib, extra).argtypes = [_vp]
     return lib
 
 

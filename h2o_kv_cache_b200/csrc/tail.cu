@@ -27,9 +27,53 @@
 #include <cstring>
 
 #include "h2o_internal.cuh"
+#include "sm100.cuh"
+
+// Phase stamps: with -DH2O_STAMPS (see h2o_kv_cache_b200/stamps.py) thread 0 of
+// the first kTailStampCtas CTAs records clock64() at the phase boundaries
+// (kernel start after the dependency wait, end of phase 1, end of the
+// selection, end of the compaction, start and end of the scatter); the
+// default build compiles every stamp to nothing.
+#ifdef H2O_STAMPS
+constexpr int kTailStampCtas = 1024, kTailStampSlots = 8;
+__device__ unsigned long long g_h2o_tail_stamps[kTailStampCtas * kTailStampSlots];
+#define H2O_TAIL_STAMP(i)                                                          \
+  do {                                                                             \
+    if (threadIdx.x == 0 && blockIdx.x < kTailStampCtas)                           \
+      g_h2o_tail_stamps[blockIdx.x * kTailStampSlots + (i)] = clock64();           \
+  } while (0)
+extern "C" int h2o_tail_stamps_read(unsigned long long* host) {
+  return cudaMemcpyFromSymbol(host, g_h2o_tail_stamps, sizeof(g_h2o_tail_stamps)) == cudaSuccess ? 0 : -1;
+}
+#else
+#define H2O_TAIL_STAMP(i) \
+  do {                    \
+  } while (0)
+#endif
 
 namespace h2o {
 namespace {
+
+using sm100::smem_u32;
+
+// Bulk (untiled) copy global -> shared of `bytes` (a multiple of 16; both
+// addresses 16-byte aligned), completing on the mbarrier `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// Waits for the phase of `parity` of a CTA-local mbarrier for at most ~1 s;
+// false on a timeout.
+__device__ __forceinline__ bool tail_wait(uint32_t bar, uint32_t parity) {
+  if (sm100::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = sm100::global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0 && sm100::global_timer_ns() - t0 > 1000000000ull) return false;
+  }
+}
 
 constexpr int kTailThreads = 512;
 constexpr int kMaxCluster = 16;
@@ -38,10 +82,11 @@ constexpr int kDigitBits = 11;                     // radix digit
 constexpr int kBins = 1 << kDigitBits;
 constexpr int kBinsPerThread = kBins / kTailThreads;
 static_assert(kBinsPerThread == 4, "one 16-byte histogram read per thread");
-// chunk rows per warp read ahead: 8 in the one-layer kernel; the grouped
-// kernel (many caches per launch) keeps 2 CTAs an SM resident instead, which
-// caps it at 64 registers a thread
-template <int L> constexpr int pre_rows() { return L == 1 ? 8 : 4; }
+// chunk rows per warp read ahead on the register path of phase 4: 8 in the
+// one-layer kernel; the grouped kernel (many caches per launch) keeps 2 CTAs an
+// SM resident instead, which caps it at 64 registers a thread, and its caches
+// are large enough for the bulk-copy path
+template <int L> constexpr int pre_rows() { return L == 1 ? 8 : 1; }
 template <int L> constexpr int min_blocks() { return L == 1 ? 1 : 2; }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -141,6 +186,7 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   __shared__ int64_t sh_kth;
   __shared__ int sh_state;                            // 0 searching, 1 found, 2 too few
   __shared__ uint32_t sh_off, sh_tot;
+  __shared__ __align__(8) uint64_t row_bar[2];        // bulk loads of chunk rows (phase 4)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthr = kTailThreads, nwarps = kTailThreads / 32;
@@ -170,13 +216,33 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   }
   // everything below reads what the preceding kernel of the stream wrote
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  H2O_TAIL_STAMP(0);
 
   // Chunk rows i = lo_s + warp + k * nwarps (k = 0, 1, ...) are this warp's to
   // scatter.  The first kPre are read now, so that their latency hides behind
   // the reduction and the selection: lane c holds vector c of the row's K
   // vectors followed by its V vectors.
   const int rv = p.row_vecs, vecs2 = 2 * rv;
-  const bool pre_ok = vecs2 <= 32;
+  // Phase 4 of the grouped kernel brings the CTA's chunk rows (contiguous in
+  // the chunk's K and V) into the keys' shared memory, free by then, with one
+  // bulk copy per batch of nb rows (two batches in flight), and the warps store
+  // them to their slots: with two CTAs an SM and 64 registers a thread it has
+  // too few registers to keep enough rows in flight on the register path.  The
+  // one-layer kernel (one CTA an SM, 8 rows a warp read at kernel start, 8 more
+  // in flight at a time) takes the register path: measured 10k cycles for the
+  // 256 rows of a 32k-slot CTA against 22k through bulk copies, 4k against 14k
+  // for the 128 rows of a 16k-slot CTA.
+  const uint32_t row_bytes = (uint32_t)rv * 16u;
+  const int64_t n_rows = hi_s > lo_s ? hi_s - lo_s : 0;
+  int nb = (int)((int64_t)p.per * 8 / (4 * (int64_t)row_bytes));
+  if (nb > 64) nb = 64;
+  const bool bulk = L > 1 && nb >= 16 && n_rows > 0;
+  if (bulk && tid == 0) {
+    sm100::mbar_init(smem_u32(&row_bar[0]), 1);
+    sm100::mbar_init(smem_u32(&row_bar[1]), 1);
+    sm100::fence_mbar_init();
+  }
+  const bool pre_ok = vecs2 <= 32 && !bulk;
   const int64_t n_mine = hi_s - lo_s > warp ? (hi_s - lo_s - warp + nwarps - 1) / nwarps : 0;
   uint4 pre[kPre];
   if (pre_ok) {
@@ -197,63 +263,91 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   int32_t* ps = p.pos + bh * M;
   const int64_t lim = p.t0 - p.R;               // eligible: 0 <= pos < t0 - R
   const bool vec = (M & 3) == 0;                // rows of scores / positions 16-byte aligned
-  for (int64_t s0 = lo + 4 * (int64_t)tid; s0 < hi; s0 += 4 * (int64_t)nthr) {
-    float scv[4] = {0.f, 0.f, 0.f, 0.f};
-    int32_t psv[4] = {-1, -1, -1, -1};
+  // Two rounds' loads are issued before either round's stores, so twice the
+  // bytes are in flight (the stores could alias the loads as far as the
+  // compiler knows, and would otherwise hold back the next round's loads).
+  struct Round {
+    float sc[4];
+    int32_t ps[4];
+    unsigned long long av[4];
+  };
+  auto load_round = [&](int64_t s0, Round& x) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x.sc[e] = 0.f;
+      x.ps[e] = -1;
+      x.av[e] = 0ull;
+    }
+    if (s0 >= hi) return;
     if (vec && s0 + 4 <= hi) {
       const float4 f = *reinterpret_cast<const float4*>(sc + s0);
       const int4 q = *reinterpret_cast<const int4*>(ps + s0);
-      scv[0] = f.x; scv[1] = f.y; scv[2] = f.z; scv[3] = f.w;
-      psv[0] = q.x; psv[1] = q.y; psv[2] = q.z; psv[3] = q.w;
+      x.sc[0] = f.x; x.sc[1] = f.y; x.sc[2] = f.z; x.sc[3] = f.w;
+      x.ps[0] = q.x; x.ps[1] = q.y; x.ps[2] = q.z; x.ps[3] = q.w;
     } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         if (s0 + e < hi) {
-          scv[e] = sc[s0 + e];
-          psv[e] = ps[s0 + e];
+          x.sc[e] = sc[s0 + e];
+          x.ps[e] = ps[s0 + e];
         }
     }
-    unsigned long long av[4] = {0ull, 0ull, 0ull, 0ull};
     if (s0 + 4 <= nv) {                         // acc rows and s0 are multiples of 4 words
-      ulonglong2* a2 = reinterpret_cast<ulonglong2*>(acc + s0);
+      const ulonglong2* a2 = reinterpret_cast<const ulonglong2*>(acc + s0);
       const ulonglong2 x0 = a2[0], x1 = a2[1];
-      av[0] = x0.x; av[1] = x0.y; av[2] = x1.x; av[3] = x1.y;
+      x.av[0] = x0.x; x.av[1] = x0.y; x.av[2] = x1.x; x.av[3] = x1.y;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (s0 + e < nv) x.av[e] = acc[s0 + e];
+    }
+  };
+  auto finish_round = [&](int64_t s0, Round& x) {
+    if (s0 >= hi) return;
+    if (s0 + 4 <= nv) {
+      ulonglong2* a2 = reinterpret_cast<ulonglong2*>(acc + s0);
       a2[0] = make_ulonglong2(0ull, 0ull);
       a2[1] = make_ulonglong2(0ull, 0ull);
     } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (s0 + e < nv) {
-          av[e] = acc[s0 + e];
-          acc[s0 + e] = 0ull;
-        }
+        if (s0 + e < nv) acc[s0 + e] = 0ull;
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int64_t s = s0 + e;
       if (s >= hi) break;
-      float v = scv[e];
-      if (s < nv) v += colsum_value(av[e], p.fx_inv);
-      scv[e] = v;
-      const int32_t q = psv[e];
+      float v = x.sc[e];
+      if (s < nv) v += colsum_value(x.av[e], p.fx_inv);
+      x.sc[e] = v;
+      const int32_t q = x.ps[e];
       keys[s - lo] = (q >= 0 && q < lim)
                          ? (p.recency ? 0ull : (uint64_t)ordered_bits(v) << 32) | (uint32_t)q
                          : kNoKey;
     }
     if (s0 < nv) {
       if (vec && s0 + 4 <= hi) {
-        *reinterpret_cast<float4*>(sc + s0) = make_float4(scv[0], scv[1], scv[2], scv[3]);
+        *reinterpret_cast<float4*>(sc + s0) = make_float4(x.sc[0], x.sc[1], x.sc[2], x.sc[3]);
       } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (s0 + e < nv) sc[s0 + e] = scv[e];
+          if (s0 + e < nv) sc[s0 + e] = x.sc[e];
       }
     }
+  };
+  for (int64_t s0 = lo + 4 * (int64_t)tid; s0 < hi; s0 += 8 * (int64_t)nthr) {
+    const int64_t s1 = s0 + 4 * (int64_t)nthr;
+    Round ra, rb;
+    load_round(s0, ra);
+    load_round(s1, rb);
+    finish_round(s0, ra);
+    finish_round(s1, rb);
   }
   for (int64_t i = lo_s + tid; i < hi_s; i += nthr) {
     ns[i - lo_s] = colsum_value(acc[M + i], p.fx_inv);
     acc[M + i] = 0ull;
   }
+  H2O_TAIL_STAMP(1);
   csync();   // rank 0's histograms are zero, every CTA has its keys
 
   // ---- 2. radix select of the need-th smallest key over the cluster,
@@ -318,20 +412,23 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
     __syncthreads();
   }
 
+  H2O_TAIL_STAMP(2);
   // ---- 3. evicted slots in ascending order, then the empty slots
   const int state = sh_state;
   const uint64_t prefix = sh_prefix, mask = sh_mask;
   const bool do_sel = need > 0 && state == 1;
-  const int64_t run = (nloc + nthr - 1) / nthr;
-  const int64_t j0 = (int64_t)tid * run, j1 = j0 + run < nloc ? j0 + run : nloc;
+  auto selected = [&](int64_t j) -> bool {
+    if (j >= nloc) return false;
+    const uint64_t key = keys[j];
+    return key != kNoKey && (key & mask) <= prefix;
+  };
+  // the CTA's count, thread t taking keys t, t + nthr, ... (a warp reads
+  // consecutive words: no shared-memory bank conflicts)
   uint32_t mine = 0;
   if (do_sel)
-    for (int64_t j = j0; j < j1; ++j) {
-      const uint64_t key = keys[j];
-      mine += (key != kNoKey && (key & mask) <= prefix) ? 1u : 0u;
-    }
+    for (int64_t j = tid; j < nloc; j += nthr) mine += selected(j) ? 1u : 0u;
   uint32_t cta_sel;
-  const uint32_t my_off = block_excl_scan(mine, warp_sum, &cta_sel);
+  (void)block_excl_scan(mine, warp_sum, &cta_sel);
   const uint32_t cnt0 = dsmem_addr(&cnt[0], 0);
   if (tid == 0) dsmem_st(cnt0 + rank * 4u, cta_sel);
   csync();
@@ -349,16 +446,31 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   int32_t* fr = p.freed + bh * S;
   int32_t* ev = p.evicted + bh * S;   // the delta record: the position each filled slot held
   if (do_sel) {
-    int64_t o = (int64_t)sh_off + my_off;
-    for (int64_t j = j0; j < j1; ++j) {
-      const uint64_t key = keys[j];
-      if (key != kNoKey && (key & mask) <= prefix) {
+    // in ascending slot order: blocks of nthr consecutive keys, a ballot per
+    // warp, the warps' counts added in warp order
+    int64_t base = sh_off;
+    for (int64_t j0 = 0; j0 < nloc; j0 += nthr) {
+      const int64_t j = j0 + tid;
+      const bool sel = selected(j);
+      const unsigned bal = __ballot_sync(0xffffffffu, sel);
+      if (lane == 0) warp_sum[warp] = (uint32_t)__popc(bal);
+      __syncthreads();
+      uint32_t off = 0, tot = 0;
+      for (int w = 0; w < nwarps; ++w) {
+        const uint32_t x = warp_sum[w];
+        off += w < warp ? x : 0u;
+        tot += x;
+      }
+      off += (uint32_t)__popc(bal & ((1u << lane) - 1u));
+      if (sel) {
+        const int64_t o = base + off;
         if (o < need) {
           fr[o] = (int32_t)(lo + j);
-          ev[o] = (int32_t)(uint32_t)key;   // the key's low word is the slot's position
+          ev[o] = (int32_t)(uint32_t)keys[j];   // the key's low word is the slot's position
         }
-        ++o;
       }
+      base += tot;
+      __syncthreads();   // warp_sum is rewritten by the next block
     }
   }
   if (rank == 0 && tid == 0 && !sel_ok) atomicOr(p.err, kErrSelect);
@@ -366,10 +478,75 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
     fr[need + e] = (int32_t)(nv + e);
     ev[need + e] = -1;
   }
+  H2O_TAIL_STAMP(3);
   csync();   // the freed list is complete; rank 0's shared memory is no longer read
+  H2O_TAIL_STAMP(4);
 
   // ---- 4. chunk row i -> slot fr[i]: K and V rows, pos = t0 + i, initial score
   if (!sel_ok) return;
+  if (bulk) {
+    const uint32_t stage = smem_u32(dyn);
+    const uint32_t half = 2u * (uint32_t)nb * row_bytes;     // a batch: nb K rows, then nb V rows
+    const int n_batches = (int)((n_rows + nb - 1) / nb);
+    const uint4* ksrc = p.k + (bh * S + lo_s) * rv;
+    const uint4* vsrc = p.v + (bh * S + lo_s) * rv;
+    auto issue = [&](int b) {
+      const int64_t r0 = (int64_t)b * nb;
+      const uint32_t nr = (uint32_t)(n_rows - r0 < nb ? n_rows - r0 : nb);
+      const uint32_t dst = stage + (uint32_t)(b & 1) * half;
+      const uint32_t bar = smem_u32(&row_bar[b & 1]);
+      sm100::mbar_arrive_expect_tx(bar, 2u * nr * row_bytes);
+      bulk_load(dst, ksrc + r0 * rv, nr * row_bytes, bar);
+      bulk_load(dst + (uint32_t)nb * row_bytes, vsrc + r0 * rv, nr * row_bytes, bar);
+    };
+    if (tid == 0) issue(0);
+    int issued = 1, waited = 0;
+    bool ok = true;
+    for (int b = 0; b < n_batches; ++b) {
+      // the other half was released by the barrier that ended batch b - 1
+      if (b + 1 < n_batches) {
+        if (tid == 0) issue(b + 1);
+        ++issued;
+      }
+      ok = __syncthreads_and(tail_wait(smem_u32(&row_bar[b & 1]), (uint32_t)(b >> 1) & 1u));
+      if (!ok) break;
+      ++waited;
+      // a warp per row: shared memory -> the row's slot, 16 bytes a lane
+      const int64_t r0 = (int64_t)b * nb;
+      const int nr = (int)(n_rows - r0 < nb ? n_rows - r0 : nb);
+      const uint4* kst = reinterpret_cast<const uint4*>(dyn + (size_t)(b & 1) * half);
+      const uint4* vst = kst + (size_t)nb * rv;
+      for (int t = warp; t < nr; t += nwarps) {
+        const int64_t i = lo_s + r0 + t;
+        const int32_t slot = ld_relaxed(fr + i);
+        if (slot < 0 || slot >= M) {
+          if (lane == 0) atomicOr(p.err, kErrBounds);
+          continue;
+        }
+        const int64_t dst = (bh * M + slot) * rv;
+        for (int c = lane; c < vecs2; c += 32) {
+          if (c < rv) p.kc[dst + c] = kst[(size_t)t * rv + c];
+          else p.vc[dst + c - rv] = vst[(size_t)t * rv + c - rv];
+        }
+        if (lane == 0) {
+          p.pos[bh * M + slot] = (int32_t)(p.t0 + i);
+          p.scores[bh * M + slot] = ns[i - lo_s];
+        }
+      }
+      __syncthreads();   // every warp is done reading this half
+    }
+    if (!ok) {
+      // a load did not land within the limit: record it, and let the loads in
+      // flight finish (again bounded) before the CTA's shared memory goes
+      if (tid == 0) atomicOr(p.err, kErrTimeout);
+      for (int b = waited; b < issued; ++b) tail_wait(smem_u32(&row_bar[b & 1]), (uint32_t)(b >> 1) & 1u);
+    }
+#ifdef H2O_STAMPS
+    __syncthreads();
+    H2O_TAIL_STAMP(5);
+#endif
+    return;
+  }
   auto finish_row = [&](int64_t i, int32_t slot) {
     if (lane == 0) {
       p.pos[bh * M + slot] = (int32_t)(p.t0 + i);
@@ -431,6 +608,10 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
       }
     }
   }
+#ifdef H2O_STAMPS
+  __syncthreads();   // every warp's rows are stored
+  H2O_TAIL_STAMP(5);
+#endif
 }
 
 size_t tail_smem(int64_t M, int64_t S, int cs, int* per, int* per_s) {

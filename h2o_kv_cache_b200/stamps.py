@@ -19,6 +19,7 @@ import tempfile
 import numpy as np
 
 KCTAS, KSLOTS = 148, 1200
+TAIL_CTAS, TAIL_SLOTS = 1024, 8
 # slot bases, as in csrc/attn_umma.cu
 ISSUE_K, K_FULL, S_EMPTY, PAIR_ISSUED, S_FULL, PAIR_END = 0, 64, 128, 256, 320, 448
 ST_START, ST_READY, OT_READY, ST_FULL, P_EMPTY, P_FULL = 512, 608, 704, 800, 896, 992
@@ -52,9 +53,26 @@ def _child(cfg_id, layers, steps, out_path):
             caches[0].step(*chunks[0][i])
     torch.cuda.synchronize()
     buf = (ctypes.c_ulonglong * (KCTAS * KSLOTS))()
-    if h2o.lib.h2o_stamps_read(buf) != 0:
-        raise RuntimeError("h2o_stamps_read failed")
-    np.save(out_path, np.frombuffer(buf, dtype=np.uint64).reshape(KCTAS, KSLOTS).astype(np.int64))
+    tbuf = (ctypes.c_ulonglong * (TAIL_CTAS * TAIL_SLOTS))()
+    if h2o.lib.h2o_stamps_read(buf) != 0 or h2o.lib.h2o_tail_stamps_read(tbuf) != 0:
+        raise RuntimeError("reading the stamps failed")
+    np.savez(out_path, attn=np.frombuffer(buf, dtype=np.uint64).reshape(KCTAS, KSLOTS).astype(np.int64),
+             tail=np.frombuffer(tbuf, dtype=np.uint64).reshape(TAIL_CTAS, TAIL_SLOTS).astype(np.int64))
+
+
+def summarize_tail(tt):
+    """Median (over CTAs) of each phase of the tail kernel, in SM clock cycles."""
+    ok = (tt[:, 0] > 0) & (tt[:, 5] > tt[:, 0])
+    if not ok.any():
+        return {}
+    t = tt[ok]
+    names = ["score accumulate and keys (phase 1)", "selection (incl. the first barrier)",
+             "compaction", "barrier before the scatter", "scatter", "whole kernel"]
+    spans = [t[:, 1] - t[:, 0], t[:, 2] - t[:, 1], t[:, 3] - t[:, 2], t[:, 4] - t[:, 3],
+             t[:, 5] - t[:, 4], t[:, 5] - t[:, 0]]
+    out = {nm: float(np.median(x)) for nm, x in zip(names, spans)}
+    out["CTAs stamped"] = float(ok.sum())
+    return out
 
 
 def summarize(st):
@@ -114,12 +132,14 @@ def main():
     sys.path.insert(0, here)
     import build as B
     lib = B.build(stamps=True)
-    out = os.path.join(tempfile.mkdtemp(), "stamps.npy")
+    out = os.path.join(tempfile.mkdtemp(), "stamps.npz")
     env = dict(os.environ, H2O_LIBRARY=lib)
     subprocess.run([sys.executable, "-m", "h2o_kv_cache_b200.stamps", "--config", str(args.config),
                     "--layers", str(args.layers), "--steps", str(args.steps), "--child", out],
                    check=True, env=env, cwd=os.path.dirname(here))
-    res = summarize(np.load(out))
+    data = np.load(out)
+    res = summarize(data["attn"])
+    res["tail (one launch: the last step's)"] = summarize_tail(data["tail"])
     print(f"workload config {args.config}, {args.layers} layer(s), last of {args.steps} steps; "
           "medians over the first wave's CTAs, SM clock cycles")
     for part, vals in res.items():

@@ -104,3 +104,12 @@ def test_injected_allocation_failure_is_reported(monkeypatch):
     assert _lib.lib.h2o_step(h, dummy, dummy, dummy, dummy, 8, None) == _lib.H2O_ESTATE
     assert _lib.lib.h2o_prefill(h, dummy, dummy, dummy, None, 1, 8, None) == _lib.H2O_ENOMEM
     assert _lib.lib.h2o_destroy(h) == _lib.H2O_OK
+
+
+def test_create_policy_rejects_unknown_policies():
+    h = ctypes.c_void_p()
+    assert _lib.lib.h2o_create_policy(64, 8, 4, 2, 64, _lib.H2O_F32, 7, ctypes.byref(h)) == _lib.H2O_EINVAL
+    assert not h.value and b"policy" in _lib.lib.h2o_last_error(None)
+    for pol in (_lib.H2O_POLICY_H2O, _lib.H2O_POLICY_LR):
+        assert _lib.lib.h2o_create_policy(64, 8, 4, 2, 64, _lib.H2O_F32, pol, ctypes.byref(h)) == _lib.H2O_OK
+        assert _lib.lib.h2o_destroy(h) == _lib.H2O_OK

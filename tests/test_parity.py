@@ -452,7 +452,8 @@ def _layer_streams(cfg, layers, T):
     return out, bounds
 
 
-@pytest.mark.parametrize("case", ["b4-3layers", "tiny-bf16-35layers", "mixed-fp32"])
+@pytest.mark.parametrize("case", ["b4-3layers", "tiny-bf16-35layers", "mixed-fp32",
+                                  "10layers-640caches"])
 def test_step_layers_matches_single_steps(h2o, monkeypatch, case):
     """h2o_step_layers gives, bit for bit, what one h2o_step per layer gives: one
     grid for all layers' attention and one for all tails (b4: three layers of the
@@ -468,9 +469,15 @@ def test_step_layers_matches_single_steps(h2o, monkeypatch, case):
     elif case == "tiny-bf16-35layers":
         cfg, n = _cfg(0, dtype=torch.bfloat16, d=128, name="tiny-bf16"), 35
         T = cfg.T
-    else:
+    elif case == "mixed-fp32":
         cfg, n = _cfg(0), 3
         T = cfg.T
+    else:
+        # 10 layers x 64 caches: at least two waves of caches, so the grouped tail
+        # runs one CTA per cache and moves the chunk rows with bulk copies
+        cfg = _cfg(0, name="grouped-bulk-tail", B=8, Hq=16, Hkv=8, d=128, M=2048, R=128,
+                   P=2048, S=256, T=2048 + 3 * 256, dtype=torch.bfloat16, planted=0.01)
+        n, T = 10, cfg.T
     streams, bounds = _layer_streams(cfg, range(n), T)
     mk = lambda: [h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype) for _ in range(n)]  # noqa: E731
     grouped, single = mk(), mk()
@@ -569,3 +576,35 @@ def test_lr_policy(h2o, case):
     heads = [(0, 2), (0, 5)] if case == "m2k-s1k" else None
     s = run_stream(h2o, cfg, heads=heads, T=T, policy="lr")
     assert s["ties"] == 0
+
+
+def test_step_layers_lr_policy_against_the_oracle(h2o):
+    """Grouped steps of lr caches: the same one-grid path, evictions by position."""
+    cfg = _cfg(1, name="lr-m2k-layers")
+    n, T = 3, cfg.P + 3 * cfg.S
+    streams, bounds = _layer_streams(cfg, [0, 1, 2], T)
+    caches = [h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype, policy="lr") for _ in range(n)]
+    G = cfg.G
+    orc = [H2OHeadOracle(cfg.M, cfg.R, G, cfg.d, "lr") for _ in range(n)]
+    b, h = 0, 3
+    for ci in range(len(bounds)):
+        if ci == 0:
+            outs = [caches[l].prefill(*streams[l][0]) for l in range(n)]
+        else:
+            outs = h2o.step_layers(caches, [s[ci][0] for s in streams], [s[ci][1] for s in streams],
+                                   [s[ci][2] for s in streams])
+        torch.cuda.synchronize()
+        for l in range(n):
+            q, k, v = (to64(x) for x in streams[l][ci])
+            ref = orc[l].step(q[b, h * G:(h + 1) * G], k[b, h], v[b, h])
+            where = f"lr layer {l} chunk {ci}"
+            check_outputs(to64(outs[l])[b, h * G:(h + 1) * G], ref, cfg.dtype, where)
+            slots, scores, pos = (x.cpu().numpy() for x in caches[l].read_state())
+            assert np.array_equal(slots[b, h], orc[l].last_freed), f"{where}: filled slots differ"
+            assert np.array_equal(pos[b, h], orc[l].pos), f"{where}: slot -> position map differs"
+            check_scores(scores[b, h], orc[l].score, orc[l].pos >= 0, where)
+            # the cache holds the most recent M tokens
+            t = bounds[ci][1]
+            assert sorted(int(x) for x in pos[b, h] if x >= 0) == list(range(max(0, t - cfg.M), t))
+    for c in caches:
+        c.close()
