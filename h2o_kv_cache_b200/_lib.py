@@ -54,10 +54,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
-    for extra in ("h2o_stamps_read", "h2o_tail_stamps_read"):   # the stamps build only (stamps.py)
+    for extra in ("h2o_stamps_read", "h2o_tail_stamps_read", "h2o_unit_stamps_read"):   # stamps build only
         if hasattr(lib, extra):
             getattr(lib, extra).restype = _i32
             getattr(lib, extra).argtypes = [_vp]
+    if hasattr(lib, "h2o_tail_empty_launch"):   # stamps build only
+        lib.h2o_tail_empty_launch.restype = _i32
+        lib.h2o_tail_empty_launch.argtypes = [_i32, _i32, _i32, _i32, _vp]
     return lib
 
 

@@ -67,9 +67,25 @@ __device__ unsigned long long g_h2o_stamps[h2o_stamps::kCtas * h2o_stamps::kSlot
 extern "C" int h2o_stamps_read(unsigned long long* host) {
   return cudaMemcpyFromSymbol(host, g_h2o_stamps, sizeof(g_h2o_stamps)) == cudaSuccess ? 0 : -1;
 }
+// every CTA (up to kUnitCtas): its SM, and the global timer at entry and exit
+namespace h2o_stamps {
+constexpr int kUnitCtas = 16384;
+}
+__device__ unsigned long long g_h2o_unit_stamps[h2o_stamps::kUnitCtas * 3];
+#define H2O_UNIT_STAMP(k, v)                                                   \
+  do {                                                                         \
+    if (threadIdx.x == 0 && blockIdx.x < h2o_stamps::kUnitCtas)                \
+      g_h2o_unit_stamps[blockIdx.x * 3 + (k)] = (v);                           \
+  } while (0)
+extern "C" int h2o_unit_stamps_read(unsigned long long* host) {
+  return cudaMemcpyFromSymbol(host, g_h2o_unit_stamps, sizeof(g_h2o_unit_stamps)) == cudaSuccess ? 0 : -1;
+}
 #else
 #define H2O_STAMP(i) \
   do {               \
+  } while (0)
+#define H2O_UNIT_STAMP(k, v) \
+  do {                       \
   } while (0)
 #endif
 // stamp slots: [0, 64) producer issues pair u's K tile; [64, 128) MMA warp sees it;
@@ -157,6 +173,14 @@ struct Group {
 template <int L>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_umma_kernel(const __grid_constant__ Group<L> grp) {
+#ifdef H2O_STAMPS
+  {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    H2O_UNIT_STAMP(0, smid);
+    H2O_UNIT_STAMP(1, global_timer_ns());
+  }
+#endif
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -668,6 +692,7 @@ attn_umma_kernel(const __grid_constant__ Group<L> grp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  H2O_UNIT_STAMP(2, global_timer_ns());
 }
 
 // ---------------------------------------------------------------- host side

@@ -141,7 +141,7 @@ struct TailArgs {
   int row_vecs;
   int per, per_s;          // set by launch_tail
 };
-// Cluster size the fused tail runs with for these sizes (16, 8, ..., 1), or 0
+// Cluster size the fused tail runs with for these sizes (1 to 16), or 0
 // if it cannot run (the caller then uses the three separate kernels); BH
 // caches in all, in the one-layer kernel or (grouped) the kernel for groups.
 int tail_cluster_size(int64_t M, int64_t S, int BH, bool grouped = false);

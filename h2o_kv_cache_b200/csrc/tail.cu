@@ -15,9 +15,10 @@
 //      form each eligible slot's 64-bit key (order-preserving score bits,
 //      token position) in shared memory; the chunk keys' summed weights are
 //      the new tokens' initial scores;
-//   2. MSD radix select, 11 bits a pass: every CTA adds its digit counts into
-//      rank 0's histogram through distributed shared memory, then all CTAs
-//      read the merged histogram and take the same decision;
+//   2. MSD radix select, 11 bits a pass: the bins are spread over the
+//      cluster's CTAs (each group of four bins has an owner); every CTA adds
+//      its digit counts into the owners' histograms through distributed shared
+//      memory, then all CTAs read the merged bins and take the same decision;
 //   3. ordered compaction: per-CTA counts are exchanged through rank 0, and
 //      each CTA writes its evicted slots at its offset, ascending;
 //   4. scatter of the CTA's chunk rows into the freed slots (the rows are read
@@ -35,12 +36,19 @@
 // selection, end of the compaction, start and end of the scatter); the
 // default build compiles every stamp to nothing.
 #ifdef H2O_STAMPS
-constexpr int kTailStampCtas = 1024, kTailStampSlots = 8;
+constexpr int kTailStampCtas = 1024, kTailStampSlots = 16;
 __device__ unsigned long long g_h2o_tail_stamps[kTailStampCtas * kTailStampSlots];
 #define H2O_TAIL_STAMP(i)                                                          \
   do {                                                                             \
     if (threadIdx.x == 0 && blockIdx.x < kTailStampCtas)                           \
       g_h2o_tail_stamps[blockIdx.x * kTailStampSlots + (i)] = clock64();           \
+  } while (0)
+// slot 6: the number of radix passes the selection took (a count, not a time);
+// slots 7-13: inside the selection's first pass, the compaction and the scatter
+#define H2O_TAIL_VALUE(i, v)                                                       \
+  do {                                                                             \
+    if (threadIdx.x == 0 && blockIdx.x < kTailStampCtas)                           \
+      g_h2o_tail_stamps[blockIdx.x * kTailStampSlots + (i)] = (v);                 \
   } while (0)
 extern "C" int h2o_tail_stamps_read(unsigned long long* host) {
   return cudaMemcpyFromSymbol(host, g_h2o_tail_stamps, sizeof(g_h2o_tail_stamps)) == cudaSuccess ? 0 : -1;
@@ -48,6 +56,9 @@ extern "C" int h2o_tail_stamps_read(unsigned long long* host) {
 #else
 #define H2O_TAIL_STAMP(i) \
   do {                    \
+  } while (0)
+#define H2O_TAIL_VALUE(i, v) \
+  do {                       \
   } while (0)
 #endif
 
@@ -103,6 +114,13 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile(
       "barrier.cluster.arrive.release.aligned;\n\t"
       "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The two halves of cluster_sync(), for work that can overlap the barrier.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // Address of `p` (a shared variable of this CTA) in the CTA of cluster rank `rank`.
 __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
@@ -170,6 +188,7 @@ template <int L>
 struct TailGroup {
   TailArgs t[L];
   int BH;
+  int stage;   // 1: each CTA copies all of its chunk rows into shared memory at the start
 };
 
 template <int L>
@@ -178,15 +197,16 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   extern __shared__ __align__(16) unsigned char dyn[];
   uint64_t* keys = reinterpret_cast<uint64_t*>(dyn);                   // [per]
   float* ns = reinterpret_cast<float*>(dyn + (size_t)grp.t[0].per * 8);   // [per_s]
-  __shared__ __align__(16) uint32_t hist[3][kBins];   // rank 0's copy is the merged one
+  __shared__ __align__(16) uint32_t hist[3][kBins];   // merged counts of the bins this CTA owns
   __shared__ __align__(16) uint32_t hloc[kBins];      // this CTA's counts of a pass
+  __shared__ uint32_t red_sum[kTailThreads / 32];
   __shared__ uint32_t cnt[kMaxCluster];               // rank 0: selected slots per rank
   __shared__ uint32_t warp_sum[kTailThreads / 32];
   __shared__ uint64_t sh_prefix, sh_mask;
   __shared__ int64_t sh_kth;
   __shared__ int sh_state;                            // 0 searching, 1 found, 2 too few
   __shared__ uint32_t sh_off, sh_tot;
-  __shared__ __align__(8) uint64_t row_bar[2];        // bulk loads of chunk rows (phase 4)
+  __shared__ __align__(8) uint64_t row_bar[2];        // bulk loads of chunk rows
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthr = kTailThreads, nwarps = kTailThreads / 32;
@@ -206,14 +226,19 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   const int64_t nloc = hi > lo ? hi - lo : 0;
   const int64_t lo_s = (int64_t)rank * p.per_s, hi_s = lo_s + p.per_s < S ? lo_s + p.per_s : S;
 
-  if (rank == 0)
-    for (int i = tid; i < 2 * kBins; i += nthr) (&hist[0][0])[i] = 0u;
+  // the first two passes' histograms and this CTA's counts start at zero; the
+  // cluster barrier that makes the zeros visible to the other CTAs' adds is
+  // split: arrived at here, waited for after phase 1, which hides its latency
+  for (int i = tid; i < 2 * kBins; i += nthr) (&hist[0][0])[i] = 0u;
+  for (int i = tid; i < kBins; i += nthr) hloc[i] = 0u;
   if (tid == 0) {
     sh_prefix = 0;
     sh_mask = 0;
     sh_kth = need;
     sh_state = need == 0 ? 1 : 0;
   }
+  __syncthreads();
+  if (cs > 1) cluster_arrive();
   // everything below reads what the preceding kernel of the stream wrote
   asm volatile("griddepcontrol.wait;" ::: "memory");
   H2O_TAIL_STAMP(0);
@@ -237,12 +262,19 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   int nb = (int)((int64_t)p.per * 8 / (4 * (int64_t)row_bytes));
   if (nb > 64) nb = 64;
   const bool bulk = L > 1 && nb >= 16 && n_rows > 0;
-  if (bulk && tid == 0) {
+  // Staged (the one-layer kernel, when the launch sized shared memory for it):
+  // the CTA's chunk K rows, then its V rows, are copied into shared memory
+  // after the keys by bulk copies of at most 16 KB completing on row_bar[0],
+  // issued when phase 1's loads are done (so they do not delay them) and
+  // landing during the selection; phase 4 then only stores them to their slots.
+  const bool staged = L == 1 && grp.stage != 0 && n_rows > 0;
+  const uint32_t stage_off = ((uint32_t)grp.t[0].per * 8u + (uint32_t)grp.t[0].per_s * 4u + 15u) & ~15u;
+  if ((bulk || staged) && tid == 0) {
     sm100::mbar_init(smem_u32(&row_bar[0]), 1);
     sm100::mbar_init(smem_u32(&row_bar[1]), 1);
     sm100::fence_mbar_init();
   }
-  const bool pre_ok = vecs2 <= 32 && !bulk;
+  const bool pre_ok = vecs2 <= 32 && !bulk && !staged;
   const int64_t n_mine = hi_s - lo_s > warp ? (hi_s - lo_s - warp + nwarps - 1) / nwarps : 0;
   uint4 pre[kPre];
   if (pre_ok) {
@@ -256,8 +288,9 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   }
 
   // ---- 1. scores += summed weights (the accumulator words are read and
-  // cleared for the next chunk); keys of the eligible slots; the chunk rows'
-  // initial scores.  Four slots a thread per round.
+  // cleared for the next chunk); keys of the eligible slots, and their counts
+  // by the selection's first digit (its first pass's histogram); the chunk
+  // rows' initial scores.  Four slots a thread per round.
   unsigned long long* acc = p.colacc + bh * p.acc_stride;
   float* sc = p.scores + bh * M;
   int32_t* ps = p.pos + bh * M;
@@ -302,8 +335,13 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
         if (s0 + e < nv) x.av[e] = acc[s0 + e];
     }
   };
+  // finish_round leaves the round's keys in x.av (kNoKey past the CTA's slots)
   auto finish_round = [&](int64_t s0, Round& x) {
-    if (s0 >= hi) return;
+    if (s0 >= hi) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x.av[e] = kNoKey;
+      return;
+    }
     if (s0 + 4 <= nv) {
       ulonglong2* a2 = reinterpret_cast<ulonglong2*>(acc + s0);
       a2[0] = make_ulonglong2(0ull, 0ull);
@@ -316,14 +354,19 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int64_t s = s0 + e;
-      if (s >= hi) break;
+      if (s >= hi) {
+        x.av[e] = kNoKey;
+        continue;
+      }
       float v = x.sc[e];
       if (s < nv) v += colsum_value(x.av[e], p.fx_inv);
       x.sc[e] = v;
       const int32_t q = x.ps[e];
-      keys[s - lo] = (q >= 0 && q < lim)
-                         ? (p.recency ? 0ull : (uint64_t)ordered_bits(v) << 32) | (uint32_t)q
-                         : kNoKey;
+      const uint64_t key = (q >= 0 && q < lim)
+                               ? (p.recency ? 0ull : (uint64_t)ordered_bits(v) << 32) | (uint32_t)q
+                               : kNoKey;
+      keys[s - lo] = key;
+      x.av[e] = key;
     }
     if (s0 < nv) {
       if (vec && s0 + 4 <= hi) {
@@ -335,24 +378,66 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
       }
     }
   };
-  for (int64_t s0 = lo + 4 * (int64_t)tid; s0 < hi; s0 += 8 * (int64_t)nthr) {
-    const int64_t s1 = s0 + 4 * (int64_t)nthr;
+  // the one-layer kernel loads the thread's first chunk-key word together with
+  // its first slots (the grouped kernel has no registers to spare for it)
+  const int64_t i_first = L == 1 ? lo_s + tid : hi_s;
+  const unsigned long long a_first = i_first < hi_s ? acc[M + i_first] : 0ull;
+  // counts of keys by their first digit, a warp's equal digits added at once
+  auto count_first_digits = [&](const unsigned long long (&k4)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool take = k4[e] != kNoKey;
+      const uint32_t digit = (uint32_t)(k4[e] >> (64 - kDigitBits));
+      const unsigned act = __ballot_sync(0xffffffffu, take);
+      if (take) {
+        const unsigned peers = __match_any_sync(act, digit);
+        if ((__ffs(peers) - 1) == lane) atomicAdd(&hloc[digit], (uint32_t)__popc(peers));
+      }
+    }
+  };
+  for (int64_t base = lo; base < hi; base += 8 * (int64_t)nthr) {   // the same trip count for every thread
+    const int64_t s0 = base + 4 * (int64_t)tid, s1 = s0 + 4 * (int64_t)nthr;
     Round ra, rb;
     load_round(s0, ra);
     load_round(s1, rb);
     finish_round(s0, ra);
     finish_round(s1, rb);
+    count_first_digits(ra.av);
+    count_first_digits(rb.av);
   }
-  for (int64_t i = lo_s + tid; i < hi_s; i += nthr) {
+  if (i_first < hi_s) {
+    ns[i_first - lo_s] = colsum_value(a_first, p.fx_inv);
+    acc[M + i_first] = 0ull;
+  }
+  for (int64_t i = L == 1 ? i_first + nthr : lo_s + tid; i < hi_s; i += nthr) {
     ns[i - lo_s] = colsum_value(acc[M + i], p.fx_inv);
     acc[M + i] = 0ull;
   }
+  if (staged && tid == 0) {
+    const uint32_t bar = smem_u32(&row_bar[0]);
+    const uint32_t bytes = (uint32_t)n_rows * row_bytes;
+    sm100::mbar_arrive_expect_tx(bar, 2u * bytes);
+    const uint32_t kdst = smem_u32(dyn) + stage_off;
+    const uint32_t vdst = kdst + (uint32_t)p.per_s * row_bytes;
+    const unsigned char* ksrc = reinterpret_cast<const unsigned char*>(p.k + (bh * S + lo_s) * rv);
+    const unsigned char* vsrc = reinterpret_cast<const unsigned char*>(p.v + (bh * S + lo_s) * rv);
+    for (uint32_t o = 0; o < bytes; o += 16384u) {
+      const uint32_t n = bytes - o < 16384u ? bytes - o : 16384u;
+      bulk_load(kdst + o, ksrc + o, n, bar);
+      bulk_load(vdst + o, vsrc + o, n, bar);
+    }
+  }
   H2O_TAIL_STAMP(1);
-  csync();   // rank 0's histograms are zero, every CTA has its keys
+  __syncthreads();                  // the CTA's keys and first-digit counts are complete
+  if (cs > 1) cluster_wait();       // every CTA's histograms are zero
+  H2O_TAIL_STAMP(7);
 
   // ---- 2. radix select of the need-th smallest key over the cluster,
   // kDigitBits a pass from the top (the last pass takes the 9 bits left)
-  const uint32_t hist0 = dsmem_addr(&hist[0][0], 0);
+  // bins [4 t, 4 t + 4) (thread t's) are owned by rank t % cs: the adds and
+  // the reads of a pass are spread over the cluster instead of all landing
+  // on one CTA's shared memory
+  const uint32_t hist_own = dsmem_addr(&hist[0][0], (uint32_t)tid % cs);
   int pass = 0;
   for (int top = 64; top > 0; top -= kDigitBits, ++pass) {
     if (sh_state != 0) break;                   // uniform: every CTA took the same decisions
@@ -360,23 +445,27 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
     const uint32_t dmask = (1u << (top - shift)) - 1u;
     const uint64_t prefix = sh_prefix, mask = sh_mask;
     const int64_t kth = sh_kth;
-    const uint32_t H = hist0 + (uint32_t)((pass % 3) * kBins * 4);
-    // counts of this CTA's keys in shared memory, then one remote add per
-    // non-empty bin into rank 0's histogram
-    for (int b = tid; b < kBins; b += nthr) hloc[b] = 0u;
-    __syncthreads();
-    for (int64_t j0 = 0; j0 < nloc; j0 += nthr) {
-      const int64_t j = j0 + tid;
-      const uint64_t key = j < nloc ? keys[j] : kNoKey;
-      const bool take = key != kNoKey && (key & mask) == prefix;
-      const uint32_t digit = (uint32_t)(key >> shift) & dmask;
-      const unsigned act = __ballot_sync(0xffffffffu, take);
-      if (take) {
-        const unsigned peers = __match_any_sync(act, digit);
-        if ((__ffs(peers) - 1) == lane) atomicAdd(&hloc[digit], (uint32_t)__popc(peers));
+    const uint32_t H = hist_own + (uint32_t)((pass % 3) * kBins * 4);
+    // counts of this CTA's keys in shared memory (the first pass's were taken
+    // in phase 1), then one remote add per non-empty bin into its owner's
+    // histogram
+    if (pass > 0) {
+      for (int b = tid; b < kBins; b += nthr) hloc[b] = 0u;
+      __syncthreads();
+      for (int64_t j0 = 0; j0 < nloc; j0 += nthr) {
+        const int64_t j = j0 + tid;
+        const uint64_t key = j < nloc ? keys[j] : kNoKey;
+        const bool take = key != kNoKey && (key & mask) == prefix;
+        const uint32_t digit = (uint32_t)(key >> shift) & dmask;
+        const unsigned act = __ballot_sync(0xffffffffu, take);
+        if (take) {
+          const unsigned peers = __match_any_sync(act, digit);
+          if ((__ffs(peers) - 1) == lane) atomicAdd(&hloc[digit], (uint32_t)__popc(peers));
+        }
       }
+      __syncthreads();
     }
-    __syncthreads();
+    if (pass == 0) H2O_TAIL_STAMP(8);
     {
       const uint4 c4 = *reinterpret_cast<const uint4*>(&hloc[kBinsPerThread * tid]);
       const uint32_t cv[4] = {c4.x, c4.y, c4.z, c4.w};
@@ -385,9 +474,9 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
         if (cv[b] != 0u) dsmem_add(H + (uint32_t)(kBinsPerThread * tid + b) * 4u, cv[b]);
     }
     // the histogram of the next pass was last read before the previous barrier
-    if (rank == 0)
-      for (int b = tid; b < kBins; b += nthr) hist[(pass + 1) % 3][b] = 0u;
+    for (int b = tid; b < kBins; b += nthr) hist[(pass + 1) % 3][b] = 0u;
     csync();
+    if (pass == 0) H2O_TAIL_STAMP(9);
     // thread t reads merged bins [kBinsPerThread * t, kBinsPerThread * (t + 1))
     const uint4 h4 = dsmem_ld4(H + (uint32_t)tid * 16u);
     const uint32_t hv[4] = {h4.x, h4.y, h4.z, h4.w};
@@ -410,28 +499,72 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
     }
     if (tid == 0 && (int64_t)total < kth) sh_state = 2;
     __syncthreads();
+    if (pass == 0) H2O_TAIL_STAMP(10);
   }
 
   H2O_TAIL_STAMP(2);
-  // ---- 3. evicted slots in ascending order, then the empty slots
+  H2O_TAIL_VALUE(6, (unsigned long long)pass);
+  // ---- 3. evicted slots in ascending order, then the empty slots.  Warp w
+  // takes a contiguous run of Q keys (Q a multiple of 32), lane l the keys l,
+  // l + 32, ... of it (a warp reads consecutive words: no shared-memory bank
+  // conflicts); the warps' counts give each warp its offset in the CTA, and
+  // the CTAs' counts, exchanged through rank 0, each CTA's offset.
   const int state = sh_state;
   const uint64_t prefix = sh_prefix, mask = sh_mask;
   const bool do_sel = need > 0 && state == 1;
   auto selected = [&](int64_t j) -> bool {
-    if (j >= nloc) return false;
     const uint64_t key = keys[j];
     return key != kNoKey && (key & mask) <= prefix;
   };
-  // the CTA's count, thread t taking keys t, t + nthr, ... (a warp reads
-  // consecutive words: no shared-memory bank conflicts)
-  uint32_t mine = 0;
-  if (do_sel)
-    for (int64_t j = tid; j < nloc; j += nthr) mine += selected(j) ? 1u : 0u;
-  uint32_t cta_sel;
-  (void)block_excl_scan(mine, warp_sum, &cta_sel);
+  // When the selection ended after its first pass (or evicts nothing), the
+  // CTA's count is already known -- its keys whose first digit is at most the
+  // chosen one, from the first pass's counts -- so it is published first and
+  // the exchange's cluster barrier overlaps the warps' counts of their runs.
+  // (Every CTA took the same decisions: the branch is uniform over the cluster.)
+  const bool early = !do_sel || pass == 1;
   const uint32_t cnt0 = dsmem_addr(&cnt[0], 0);
-  if (tid == 0) dsmem_st(cnt0 + rank * 4u, cta_sel);
-  csync();
+  if (early) {
+    uint32_t c = 0;
+    if (do_sel) {
+      const uint32_t bsel = (uint32_t)(prefix >> (64 - kDigitBits));
+      const uint32_t b0 = (uint32_t)(kBinsPerThread * tid);
+      const uint4 c4 = *reinterpret_cast<const uint4*>(&hloc[b0]);
+      c = (b0 <= bsel ? c4.x : 0u) + (b0 + 1 <= bsel ? c4.y : 0u) + (b0 + 2 <= bsel ? c4.z : 0u) +
+          (b0 + 3 <= bsel ? c4.w : 0u);
+    }
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (lane == 0) red_sum[warp] = c;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t t = 0;
+      for (int w = 0; w < nwarps; ++w) t += red_sum[w];
+      dsmem_st(cnt0 + rank * 4u, t);
+    }
+    if (cs > 1) cluster_arrive();
+  }
+  H2O_TAIL_STAMP(13);
+  const int64_t Q = ((nloc + nwarps - 1) / nwarps + 31) & ~(int64_t)31;
+  const int64_t w_lo = (int64_t)warp * Q;
+  const int64_t w_hi = w_lo + Q < nloc ? w_lo + Q : nloc;
+  uint32_t wcnt = 0;
+  if (do_sel)
+    for (int64_t j0 = w_lo; j0 < w_hi; j0 += 32)
+      wcnt += (uint32_t)__popc(__ballot_sync(0xffffffffu, j0 + lane < w_hi && selected(j0 + lane)));
+  if (lane == 0) warp_sum[warp] = wcnt;
+  __syncthreads();
+  uint32_t woff = 0, cta_sel = 0;
+  for (int w = 0; w < nwarps; ++w) {
+    const uint32_t x = warp_sum[w];
+    woff += w < warp ? x : 0u;
+    cta_sel += x;
+  }
+  if (!early) {
+    if (tid == 0) dsmem_st(cnt0 + rank * 4u, cta_sel);
+    if (cs > 1) cluster_arrive();
+  }
+  H2O_TAIL_STAMP(11);
+  if (cs > 1) cluster_wait();
+  else __syncthreads();
   if (warp == 0) {
     const uint32_t x = lane < (int)cs ? dsmem_ld(cnt0 + (uint32_t)lane * 4u) : 0u;
     const uint32_t off = __reduce_add_sync(0xffffffffu, lane < (int)rank ? x : 0u);
@@ -446,31 +579,19 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   int32_t* fr = p.freed + bh * S;
   int32_t* ev = p.evicted + bh * S;   // the delta record: the position each filled slot held
   if (do_sel) {
-    // in ascending slot order: blocks of nthr consecutive keys, a ballot per
-    // warp, the warps' counts added in warp order
-    int64_t base = sh_off;
-    for (int64_t j0 = 0; j0 < nloc; j0 += nthr) {
-      const int64_t j = j0 + tid;
-      const bool sel = selected(j);
+    int64_t base = (int64_t)sh_off + woff;
+    for (int64_t j0 = w_lo; j0 < w_hi; j0 += 32) {
+      const int64_t j = j0 + lane;
+      const bool sel = j < w_hi && selected(j);
       const unsigned bal = __ballot_sync(0xffffffffu, sel);
-      if (lane == 0) warp_sum[warp] = (uint32_t)__popc(bal);
-      __syncthreads();
-      uint32_t off = 0, tot = 0;
-      for (int w = 0; w < nwarps; ++w) {
-        const uint32_t x = warp_sum[w];
-        off += w < warp ? x : 0u;
-        tot += x;
-      }
-      off += (uint32_t)__popc(bal & ((1u << lane) - 1u));
       if (sel) {
-        const int64_t o = base + off;
+        const int64_t o = base + __popc(bal & ((1u << lane) - 1u));
         if (o < need) {
           fr[o] = (int32_t)(lo + j);
           ev[o] = (int32_t)(uint32_t)keys[j];   // the key's low word is the slot's position
         }
       }
-      base += tot;
-      __syncthreads();   // warp_sum is rewritten by the next block
+      base += __popc(bal);
     }
   }
   if (rank == 0 && tid == 0 && !sel_ok) atomicOr(p.err, kErrSelect);
@@ -479,10 +600,52 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
     ev[need + e] = -1;
   }
   H2O_TAIL_STAMP(3);
-  csync();   // the freed list is complete; rank 0's shared memory is no longer read
+  csync();   // the freed list is complete; no CTA's shared memory is read remotely any more
   H2O_TAIL_STAMP(4);
 
   // ---- 4. chunk row i -> slot fr[i]: K and V rows, pos = t0 + i, initial score
+  if (staged) {
+    // every copy has landed before the CTA goes on, or leaves
+    if (!__syncthreads_and(tail_wait(smem_u32(&row_bar[0]), 0u))) {
+      if (tid == 0) atomicOr(p.err, kErrTimeout);
+      tail_wait(smem_u32(&row_bar[0]), 0u);   // once more (bounded) before the shared memory goes
+      return;
+    }
+    H2O_TAIL_STAMP(12);
+    if (!sel_ok) return;
+    // a warp per row (rows warp, warp + nwarps, ...): shared memory -> the
+    // row's slot, 16 bytes a lane; lane u fetches the slot of the warp's u-th
+    // row, so one load latency covers 32 rows
+    const uint4* kst = reinterpret_cast<const uint4*>(dyn + stage_off);
+    const uint4* vst = kst + (size_t)p.per_s * rv;
+    for (int64_t k0 = 0; k0 < n_mine; k0 += 32) {
+      const int32_t my_slot = k0 + lane < n_mine ? ld_relaxed(fr + lo_s + warp + (k0 + lane) * nwarps) : -1;
+      const int kn = n_mine - k0 < 32 ? (int)(n_mine - k0) : 32;
+      for (int u = 0; u < kn; ++u) {
+        const int64_t t = warp + (k0 + u) * nwarps;
+        const int64_t i = lo_s + t;
+        const int32_t slot = __shfl_sync(0xffffffffu, my_slot, u);
+        if (slot < 0 || slot >= M) {
+          if (lane == 0) atomicOr(p.err, kErrBounds);
+          continue;
+        }
+        const int64_t dst = (bh * M + slot) * rv;
+        for (int c = lane; c < vecs2; c += 32) {
+          if (c < rv) p.kc[dst + c] = kst[(size_t)t * rv + c];
+          else p.vc[dst + c - rv] = vst[(size_t)t * rv + c - rv];
+        }
+        if (lane == 0) {
+          p.pos[bh * M + slot] = (int32_t)(p.t0 + i);
+          p.scores[bh * M + slot] = ns[i - lo_s];
+        }
+      }
+    }
+#ifdef H2O_STAMPS
+    __syncthreads();
+    H2O_TAIL_STAMP(5);
+#endif
+    return;
+  }
   if (!sel_ok) return;
   if (bulk) {
     const uint32_t stage = smem_u32(dyn);
@@ -657,7 +820,7 @@ int tail_cluster_size(int64_t M, int64_t S, int BH, bool grouped) {
   int best = 0;
   double best_cost = 1e300;
   int64_t best_waves = INT64_MAX;
-  for (int cs = kMaxCluster; cs >= 1; cs >>= 1) {
+  for (int cs = kMaxCluster; cs >= 1; --cs) {
     if (cs > 1 && M < 32LL * cs) continue;       // at least 32 slots a CTA
     int per, per_s;
     const size_t smem = tail_smem(M, S, cs, &per, &per_s);
@@ -710,6 +873,17 @@ cudaError_t launch_tail_t(const TailArgs* a, int n, int BH, int cs, bool pdl, cu
     smem = tail_smem(a[l].M, a[l].S, cs, &g.t[l].per, &g.t[l].per_s);
   }
   if (smem > kTailSmemMax) return cudaErrorInvalidValue;
+  // the one-layer kernel stages each CTA's chunk rows (K and V) in shared
+  // memory when they fit
+  g.stage = 0;
+  if (L == 1) {
+    const size_t at = (smem + 15) & ~(size_t)15;
+    const size_t rows = 2 * (size_t)g.t[0].per_s * (size_t)a[0].row_vecs * 16;
+    if (at + rows <= kTailSmemMax) {
+      smem = at + rows;
+      g.stage = 1;
+    }
+  }
   cudaError_t e = cudaFuncSetAttribute(tail_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -734,7 +908,7 @@ cudaError_t launch_tail_t(const TailArgs* a, int n, int BH, int cs, bool pdl, cu
 int tail_max_group() { return kMaxGroup; }
 
 cudaError_t launch_tail_group(const TailArgs* a, int n, int BH, int cs, bool pdl, cudaStream_t st) {
-  if (cs < 1 || cs > kMaxCluster || (cs & (cs - 1)) != 0 || n < 1 || n > kMaxGroup)
+  if (cs < 1 || cs > kMaxCluster || n < 1 || n > kMaxGroup)
     return cudaErrorInvalidValue;
   for (int l = 1; l < n; ++l)
     if (a[l].M != a[0].M || a[l].S != a[0].S) return cudaErrorInvalidValue;
@@ -746,3 +920,35 @@ cudaError_t launch_tail(const TailArgs& a, int BH, int cs, bool pdl, cudaStream_
 }
 
 }  // namespace h2o
+
+#ifdef H2O_STAMPS
+// The launch floor of the tail's launch shape: a kernel of the same block size,
+// cluster size, grid and dynamic shared memory that does nothing but the
+// dependency wait (stamps.py times it between CUDA events after a busy kernel).
+namespace {
+__global__ void __launch_bounds__(h2o::kTailThreads) tail_empty_kernel() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+}  // namespace
+extern "C" int h2o_tail_empty_launch(int cs, int grid, int smem, int pdl, void* stream) {
+  if (cs < 1 || cs > h2o::kMaxCluster || grid < cs || grid % cs != 0 || smem < 0) return -1;
+  if (cudaFuncSetAttribute(tail_empty_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncSetAttribute(tail_empty_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    return -1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(h2o::kTailThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)cs;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, tail_empty_kernel) == cudaSuccess ? 0 : -1;
+}
+#endif
