@@ -27,9 +27,9 @@
 // partials of its 256 / kc rows.  Column sums need no exchange: every key
 // belongs to one CTA.  Small chunks (S = 128: two-heads units are few) and
 // grids that would leave a partial last wave use kc > 1.
-// Exact probabilities mean O needs no rescaling.  Every MMA has N = 256: with
-// both operands in shared memory that is what keeps the tensor core near its
-// peak (N = 128 runs at about 70% of it).
+// Exact probabilities mean O needs no rescaling.  Every MMA has N = 256, the
+// widest one CTA issues: a key tile takes the fewest MMA instructions and
+// commits.
 //
 // Warp roles (320 threads): warp 0 issues TMA loads (one thread), warp 1
 // allocates TMEM and issues the MMAs (one thread), warps 2-5 / 6-9 are two
