@@ -69,6 +69,14 @@ struct h2o_ctx {
   DevBuf st_q[2], st_k[2], st_v[2], st_out;
   cudaStream_t copy_st = nullptr;
   cudaEvent_t ev_in[2] = {}, ev_free[2] = {};
+  // grouped steps led by this handle with host outputs: the layers run in
+  // sub-groups of kOutLayers, and each sub-group's outputs are copied to the
+  // host on d2h_st while the next sub-group computes (ev_sub: re-recorded after
+  // each sub-group's kernels; ev_d2h: every copy is done, waited for by the
+  // caller's stream)
+  static constexpr int kOutLayers = 4;
+  cudaStream_t d2h_st = nullptr;
+  cudaEvent_t ev_sub = nullptr, ev_d2h = nullptr;
   bool st_used[2] = {false, false};
   int st_set = 0;
   cudaEvent_t err_ev = nullptr;   // recorded after each step
@@ -224,6 +232,7 @@ struct ChunkRun {
   void* dout = nullptr;
   void* out = nullptr;          // the caller's output (host memory when hout)
   bool hout = false, host_in = false;
+  bool out_copied = false;      // the host output's copy was enqueued by run_layers
   bool decode = false, stream = false;
   int fx_shift = 0;
   h2o::StreamPlan pl;
@@ -484,7 +493,8 @@ int finish_chunk(ChunkRun& r, cudaStream_t st) {
     h->st_used[set] = true;
     h->st_set = set ^ 1;
   }
-  if (r.hout) H2O_CUDA(h, cudaMemcpyAsync(r.out, r.dout, r.q_bytes, cudaMemcpyDefault, st), "copy out");
+  if (r.hout && !r.out_copied)
+    H2O_CUDA(h, cudaMemcpyAsync(r.out, r.dout, r.q_bytes, cudaMemcpyDefault, st), "copy out");
   // the error word is read once this event has completed (by the next call)
   H2O_CUDA(h, cudaEventRecord(h->err_ev, st), "event");
   h->err_pending = true;
@@ -558,26 +568,61 @@ int run_layers(h2o_ctx** hs, int n, const void* const* q, const void* const* k,
       aa[(size_t)l] = runs[(size_t)l].a;
       ta[(size_t)l] = tail_args(runs[(size_t)l]);
     }
-    for (int l0 = 0; l0 < n; l0 += ga) {
-      const int m = n - l0 < ga ? n - l0 : ga;
-      cudaError_t e = h2o::launch_attn_umma_group(aa.data() + l0, m, true, st);
-      if (e != cudaSuccess) return cuda_fail(h0, e, "grouped attention launch");
-      runs[(size_t)l0].launches += 1;
+    // With host outputs (and no per-kernel profiling, whose events need one
+    // attention and one tail stretch) the layers run in sub-groups of
+    // kOutLayers consecutive layers, each its attention then its tail
+    // launches, and each sub-group's outputs go to the host on d2h_st while
+    // the later sub-groups compute; the caller's stream then waits for the
+    // copies, so the outputs are in host memory once it has passed the step.
+    bool any_hout = false;
+    for (int l = 0; l < n; ++l) any_hout = any_hout || runs[(size_t)l].hout;
+    const int per_sub = (any_hout && !prof && n >= 2 * h2o_ctx::kOutLayers) ? h2o_ctx::kOutLayers : n;
+    const int n_sub = (n + per_sub - 1) / per_sub;
+    if (n_sub > 1 && !h0->d2h_st) {
+      H2O_CUDA(h0, cudaStreamCreateWithFlags(&h0->d2h_st, cudaStreamNonBlocking), "copy stream");
+      H2O_CUDA(h0, cudaEventCreateWithFlags(&h0->ev_sub, cudaEventDisableTiming), "event");
+      H2O_CUDA(h0, cudaEventCreateWithFlags(&h0->ev_d2h, cudaEventDisableTiming), "event");
     }
-    if (prof) H2O_CUDA(h0, cudaEventRecord(evs[1], st), "event");
-    if (h0->grp_tail_S != S || h0->grp_tail_n != n) {
-      const int m = n < gt ? n : gt;
+    // the tail's cluster size for grouped launches of per_sub layers
+    if (h0->grp_tail_S != S || h0->grp_tail_n != per_sub) {
+      const int m = per_sub < gt ? per_sub : gt;
       h0->grp_tail_cs = m > 1 ? h2o::tail_cluster_size(h0->M, S, m * BH, true) : h0->tail_cs;
       h0->grp_tail_S = S;
-      h0->grp_tail_n = n;
+      h0->grp_tail_n = per_sub;
     }
-    for (int l0 = 0; l0 < n; l0 += gt) {
-      const int m = n - l0 < gt ? n - l0 : gt;
-      const int cs = m > 1 ? h0->grp_tail_cs : h0->tail_cs;
-      if (cs < 1) return fail(h0, H2O_ECUDA, "grouped tail: no cluster size fits");
-      cudaError_t e = h2o::launch_tail_group(ta.data() + l0, m, BH, cs, true, st);
-      if (e != cudaSuccess) return cuda_fail(h0, e, "grouped tail launch");
-      runs[(size_t)l0].launches += 1;
+    for (int g = 0; g < n_sub; ++g) {
+      const int s0 = g * per_sub, s1 = s0 + per_sub < n ? s0 + per_sub : n;
+      if (s0 >= s1) break;
+      for (int l0 = s0; l0 < s1; l0 += ga) {
+        const int m = s1 - l0 < ga ? s1 - l0 : ga;
+        cudaError_t e = h2o::launch_attn_umma_group(aa.data() + l0, m, true, st);
+        if (e != cudaSuccess) return cuda_fail(h0, e, "grouped attention launch");
+        runs[(size_t)l0].launches += 1;
+      }
+      if (prof) H2O_CUDA(h0, cudaEventRecord(evs[1], st), "event");
+      for (int l0 = s0; l0 < s1; l0 += gt) {
+        const int m = s1 - l0 < gt ? s1 - l0 : gt;
+        const int cs = m > 1 ? h0->grp_tail_cs : h0->tail_cs;
+        if (cs < 1) return fail(h0, H2O_ECUDA, "grouped tail: no cluster size fits");
+        cudaError_t e = h2o::launch_tail_group(ta.data() + l0, m, BH, cs, true, st);
+        if (e != cudaSuccess) return cuda_fail(h0, e, "grouped tail launch");
+        runs[(size_t)l0].launches += 1;
+      }
+      if (n_sub > 1) {
+        // (the wait takes the event's latest record: one event serves every sub-group)
+        H2O_CUDA(h0, cudaEventRecord(h0->ev_sub, st), "event");
+        H2O_CUDA(h0, cudaStreamWaitEvent(h0->d2h_st, h0->ev_sub, 0), "event wait");
+        for (int l = s0; l < s1; ++l) {
+          ChunkRun& r = runs[(size_t)l];
+          if (!r.hout) continue;
+          H2O_CUDA(h0, cudaMemcpyAsync(r.out, r.dout, r.q_bytes, cudaMemcpyDefault, h0->d2h_st), "copy out");
+          r.out_copied = true;
+        }
+      }
+    }
+    if (n_sub > 1) {
+      H2O_CUDA(h0, cudaEventRecord(h0->ev_d2h, h0->d2h_st), "event");
+      H2O_CUDA(h0, cudaStreamWaitEvent(st, h0->ev_d2h, 0), "event wait");
     }
   }
   if (rc != H2O_OK) return rc;
@@ -848,6 +893,9 @@ int h2o_destroy(h2o_t h) {
     if (h->ev_free[i]) cudaEventDestroy(h->ev_free[i]);
   }
   if (h->copy_st) cudaStreamDestroy(h->copy_st);
+  if (h->ev_sub) cudaEventDestroy(h->ev_sub);
+  if (h->ev_d2h) cudaEventDestroy(h->ev_d2h);
+  if (h->d2h_st) cudaStreamDestroy(h->d2h_st);
   release_state(h);
   delete h;
   return H2O_OK;

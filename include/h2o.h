@@ -38,10 +38,14 @@
  * device buffers with stream-ordered copies.  The caller owns all of them.
  * Host inputs of a step are copied on a stream of the handle's own into one of
  * two staging sets, so that they overlap the previous step's kernels; the
- * step's kernels wait for them.  Like device buffers, host buffers may be
- * reused (inputs) or read (out) once `stream` has passed the step (e.g. after
- * cudaStreamSynchronize(stream)); with pageable memory the CUDA runtime may
- * make the copies synchronous.
+ * step's kernels wait for them.  A grouped step (h2o_step_layers) of at least
+ * eight layers with host outputs runs its layers in sub-groups of four and
+ * copies each sub-group's outputs to the host on a stream of its own while the
+ * later sub-groups compute.  Like device buffers, host buffers may be reused
+ * (inputs) or read (out) once `stream` has passed the step (e.g. after
+ * cudaStreamSynchronize(stream)): the step's last work on `stream` waits for
+ * every output copy.  With pageable memory the CUDA runtime may make the
+ * copies synchronous.
  * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream); every
  * call only enqueues work on it, except where stated.  A handle is not
  * thread-safe.

@@ -504,6 +504,37 @@ def test_step_layers_matches_single_steps(h2o, monkeypatch, case):
         c.close()
 
 
+def test_step_layers_host_buffers_match_device_buffers(h2o, monkeypatch):
+    """Grouped steps with host buffers (pinned, then pageable) give, bit for bit,
+    what the same steps with device buffers give.  With host outputs and at least
+    eight layers the step runs its layers in sub-groups, each sub-group's outputs
+    copied to the host while the next one computes; the outputs are complete once
+    the caller's stream has passed the step."""
+    monkeypatch.setenv("H2O_ATTN_SPLIT", "1")
+    cfg, n = _cfg(0, dtype=torch.bfloat16, d=128, name="tiny-bf16"), 10
+    streams, bounds = _layer_streams(cfg, range(n), cfg.T)
+    mk = lambda: [h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype) for _ in range(n)]  # noqa: E731
+    dev, host = mk(), mk()
+    for l in range(n):
+        dev[l].prefill(*streams[l][0])
+        host[l].prefill(*streams[l][0])
+    for ci in range(1, len(bounds)):
+        outs_d = h2o.step_layers(dev, [s[ci][0] for s in streams], [s[ci][1] for s in streams],
+                                 [s[ci][2] for s in streams])
+        pin = ci % 2 == 1
+        hs = [tuple(x.cpu().pin_memory() if pin else x.cpu() for x in s[ci]) for s in streams]
+        houts = [torch.empty_like(h[0]).pin_memory() if pin else torch.empty_like(h[0]) for h in hs]
+        h2o.step_layers(host, [h[0] for h in hs], [h[1] for h in hs], [h[2] for h in hs], outs=houts)
+        torch.cuda.synchronize()
+        for l in range(n):
+            assert torch.equal(outs_d[l].cpu(), houts[l]), f"chunk {ci} layer {l}: outputs differ"
+            for x, y in zip(dev[l].read_state() + dev[l].read_delta(),
+                            host[l].read_state() + host[l].read_delta()):
+                assert torch.equal(x, y), f"chunk {ci} layer {l}: state differs"
+    for c in dev + host:
+        c.close()
+
+
 def test_step_layers_against_the_oracle(h2o):
     """Three layers of the 28-layer workload stepped together; sampled (batch,
     KV head) caches of each layer followed by the oracle along the stream."""
