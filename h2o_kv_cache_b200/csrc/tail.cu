@@ -25,6 +25,7 @@
 //      at the start, so only the stores remain here), recording the position
 //      each slot held before: with the freed list, the chunk's buffer delta.
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 
 #include "h2o_internal.cuh"
@@ -787,6 +788,13 @@ size_t tail_smem(int64_t M, int64_t S, int cs, int* per, int* per_s) {
 
 constexpr size_t kTailSmemMax = 180 * 1024;   // plus about 41 KB static
 
+// H2O_TAIL_STAGE=0 keeps the one-layer kernel's chunk rows out of shared memory
+// (the register path that rows too large to stage take; same results).
+bool tail_stage_enabled() {
+  const char* s = getenv("H2O_TAIL_STAGE");
+  return !(s && s[0] == '0');
+}
+
 }  // namespace
 
 int tail_cluster_size(int64_t M, int64_t S, int BH, bool grouped) {
@@ -876,7 +884,7 @@ cudaError_t launch_tail_t(const TailArgs* a, int n, int BH, int cs, bool pdl, cu
   // the one-layer kernel stages each CTA's chunk rows (K and V) in shared
   // memory when they fit
   g.stage = 0;
-  if (L == 1) {
+  if (L == 1 && tail_stage_enabled()) {
     const size_t at = (smem + 15) & ~(size_t)15;
     const size_t rows = 2 * (size_t)g.t[0].per_s * (size_t)a[0].row_vecs * 16;
     if (at + rows <= kTailSmemMax) {

@@ -340,15 +340,19 @@ def test_host_buffers_match_device_buffers(h2o):
     b.close()
 
 
+@pytest.mark.parametrize("stage", ["1", "0"])
 @pytest.mark.parametrize("base,kw,T", [
     (0, {}, None),
     (0, {"dtype": torch.bfloat16, "d": 128, "M": 301, "R": 45, "P": 203, "S": 37}, 203 + 6 * 37 + 11),
     (1, {}, 2048 + 3 * 1024),
 ])
-def test_fused_tail_matches_split_kernels(h2o, monkeypatch, base, kw, T):
-    """The fused cluster tail and the three separate kernels sum the partial
-    rows in the same order, so outputs, state and cache agree bit for bit."""
+def test_fused_tail_matches_split_kernels(h2o, monkeypatch, base, kw, T, stage):
+    """The fused cluster tail and the three separate kernels accumulate the
+    summed weights the same way, so outputs, state and cache agree bit for bit;
+    the fused kernel with its chunk rows staged in shared memory, and without
+    (H2O_TAIL_STAGE=0: the register path that rows too large to stage take)."""
     from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    monkeypatch.setenv("H2O_TAIL_STAGE", stage)
     cfg = _cfg(base, **kw)
     T = cfg.T if T is None else T
     Q, K, V = gen_batch(cfg, 0, device="cuda", T=T)
