@@ -13,16 +13,17 @@
 //   1. add the summed weights (the fixed-point accumulator row the attention
 //      kernel filled, read once and cleared) to the scores of its slots, and
 //      form each eligible slot's 64-bit key (order-preserving score bits,
-//      token position) in shared memory; the chunk keys' summed weights are
-//      the new tokens' initial scores;
+//      token position) in shared memory, counting the keys by their first
+//      radix digit on the way; the chunk keys' summed weights are the new
+//      tokens' initial scores;
 //   2. MSD radix select, 11 bits a pass: the bins are spread over the
 //      cluster's CTAs (each group of four bins has an owner); every CTA adds
 //      its digit counts into the owners' histograms through distributed shared
 //      memory, then all CTAs read the merged bins and take the same decision;
 //   3. ordered compaction: per-CTA counts are exchanged through rank 0, and
 //      each CTA writes its evicted slots at its offset, ascending;
-//   4. scatter of the CTA's chunk rows into the freed slots (the rows are read
-//      at the start, so only the stores remain here), recording the position
+//   4. scatter of the CTA's chunk rows into the freed slots (the rows were
+//      read earlier, so mostly stores remain here), recording the position
 //      each slot held before: with the freed list, the chunk's buffer delta.
 #include <cstdint>
 #include <cstdlib>
@@ -244,20 +245,23 @@ __global__ void __launch_bounds__(kTailThreads, min_blocks<L>()) tail_kernel(con
   asm volatile("griddepcontrol.wait;" ::: "memory");
   H2O_TAIL_STAMP(0);
 
-  // Chunk rows i = lo_s + warp + k * nwarps (k = 0, 1, ...) are this warp's to
-  // scatter.  The first kPre are read now, so that their latency hides behind
-  // the reduction and the selection: lane c holds vector c of the row's K
-  // vectors followed by its V vectors.
+  // The CTA's chunk rows reach phase 4 one of three ways.
+  //  - Staged (the one-layer kernel when they fit; see below): bulk-copied into
+  //    shared memory after phase 1.
+  //  - Bulk (the grouped kernel): phase 4 copies them into the keys' shared
+  //    memory, free by then, one bulk copy per batch of nb rows (two batches in
+  //    flight), and the warps store them to their slots; with two CTAs an SM
+  //    and 64 registers a thread it could not keep enough rows in flight in
+  //    registers.
+  //  - Registers (rows too large to stage): chunk rows i = lo_s + warp +
+  //    k * nwarps (k = 0, 1, ...) are this warp's to scatter, the first kPre
+  //    read now so that their latency hides behind phases 1-3 (lane c holds
+  //    vector c of the row's K vectors followed by its V vectors), then 8 rows
+  //    a warp in flight at a time.
+  // Measured at 32k/2k (8 caches): phase 4 took 10.2k cycles from registers and
+  // 22k through bulk copies in phase 4 for a CTA's 256 rows (clusters of 8),
+  // and staged 8.1k for its 205 rows (clusters of 10).
   const int rv = p.row_vecs, vecs2 = 2 * rv;
-  // Phase 4 of the grouped kernel brings the CTA's chunk rows (contiguous in
-  // the chunk's K and V) into the keys' shared memory, free by then, with one
-  // bulk copy per batch of nb rows (two batches in flight), and the warps store
-  // them to their slots: with two CTAs an SM and 64 registers a thread it has
-  // too few registers to keep enough rows in flight on the register path.  The
-  // one-layer kernel (one CTA an SM, 8 rows a warp read at kernel start, 8 more
-  // in flight at a time) takes the register path: measured 10k cycles for the
-  // 256 rows of a 32k-slot CTA against 22k through bulk copies, 4k against 14k
-  // for the 128 rows of a 16k-slot CTA.
   const uint32_t row_bytes = (uint32_t)rv * 16u;
   const int64_t n_rows = hi_s > lo_s ? hi_s - lo_s : 0;
   int nb = (int)((int64_t)p.per * 8 / (4 * (int64_t)row_bytes));
