@@ -803,6 +803,10 @@ bool tail_stage_enabled() {
 
 int tail_cluster_size(int64_t M, int64_t S, int BH, bool grouped) {
   static_assert(kMaxCluster == 16, "cluster sizes below assume 16");
+  // H2O_TAIL_CS=k asks for clusters of k CTAs (used when that size fits and can
+  // be scheduled; otherwise the choice below stands)
+  const char* fs = getenv("H2O_TAIL_CS");
+  const int forced = fs ? atoi(fs) : 0;
   if (cudaFuncSetAttribute(tail_kernel<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
       cudaFuncSetAttribute(tail_kernel<kMaxGroup>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
@@ -812,7 +816,7 @@ int tail_cluster_size(int64_t M, int64_t S, int BH, bool grouped) {
   // at least two waves of them.  The CTAs then need no cluster barriers, and
   // with two CTAs an SM and more caches than CTA slots the launch streams its
   // bytes at the HBM rate instead of waiting on barrier latency.
-  if (grouped) {
+  if (grouped && forced < 1) {
     int per, per_s;
     const size_t smem = tail_smem(M, S, 1, &per, &per_s);
     int n = 0;
@@ -860,6 +864,7 @@ int tail_cluster_size(int64_t M, int64_t S, int BH, bool grouped) {
       n = 0;
     }
     if (n < 1) continue;
+    if (cs == forced) return cs;
     const int64_t waves = (BH + n - 1) / n;
     const double cost = (double)waves / cs;
     if (cost < best_cost * (1 - 1e-9) || (cost <= best_cost * (1 + 1e-9) && waves < best_waves)) {

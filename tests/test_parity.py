@@ -383,6 +383,35 @@ def test_fused_tail_matches_split_kernels(h2o, monkeypatch, base, kw, T, stage):
     split.close()
 
 
+def test_fused_tail_every_cluster_size(h2o, monkeypatch):
+    """The fused tail at cluster sizes 1 to 16 (H2O_TAIL_CS), powers of two or
+    not, agrees bit for bit with the three separate kernels: per-CTA slot and
+    chunk-row ranges that do not divide M and S, histogram bins owned by rank
+    t mod cs, the per-rank counts of the ordered compaction."""
+    from h2o_kv_cache_b200.workload import gen_batch, split_chunks
+    cfg = _cfg(0, dtype=torch.bfloat16, d=128, B=1, Hq=8, Hkv=4, M=1000, R=64, P=1000, S=96,
+               T=1000 + 4 * 96 + 17)
+    Q, K, V = gen_batch(cfg, 0, device="cuda")
+    chunks = split_chunks(Q, K, V, cfg.bounds())
+    monkeypatch.setenv("H2O_SPLIT_TAIL", "1")
+    ref = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+    want = [ref.prefill(*chunks[0])] + [ref.step(*c) for c in chunks[1:]]
+    torch.cuda.synchronize()
+    want_state = [x.clone() for x in ref.read_state() + ref.read_delta() + ref.read_kv()]
+    ref.close()
+    monkeypatch.delenv("H2O_SPLIT_TAIL")
+    for cs in (1, 2, 3, 5, 7, 10, 13, 16):
+        monkeypatch.setenv("H2O_TAIL_CS", str(cs))
+        c = h2o.H2OCache(cfg.M, cfg.R, cfg.Hq, cfg.Hkv, cfg.d, cfg.dtype)
+        got = [c.prefill(*chunks[0])] + [c.step(*ch) for ch in chunks[1:]]
+        torch.cuda.synchronize()
+        for ci, (a, b) in enumerate(zip(got, want)):
+            assert torch.equal(a, b), f"clusters of {cs}, chunk {ci}: outputs differ"
+        for x, y in zip(c.read_state() + c.read_delta() + c.read_kv(), want_state):
+            assert torch.equal(x, y), f"clusters of {cs}: state differs"
+        c.close()
+
+
 def test_standalone_select_with_ties(h2o):
     rng = np.random.default_rng(11)
     for trial in range(12):
