@@ -88,3 +88,51 @@ def test_reference_arm_maps_no_product_library():
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip().splitlines()[-1] == "CLEAN"
+
+
+def test_roofline_objects_arithmetic():
+    # achieved = algorithmic FLOPs (bytes) per launch / the launch's time; the
+    # 28-layer workload is read against the sustained peak, one layer against
+    # the burst peak
+    from h2o_kv_cache_b200.workload import CONFIGS
+    b = _bench()
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "source": "measured"}
+    res = {"flops": 700e9, "attn_ms": 1.0, "sel_ms": 0.01}
+    for cid, peak in ((4, 1400.0), (1, 1600.0)):
+        cfg = CONFIGS[cid]
+        att, sel = b.roofline_objects(cfg, res, peaks)
+        assert att["achieved"] == pytest.approx(700.0)
+        assert att["peak"] == peak and att["frac"] == pytest.approx(700.0 / peak)
+        assert att["frac_of_burst_peak"] == pytest.approx(700.0 / 1600.0)
+        gbs = b.select_scatter_bytes(cfg, cfg.S) / 1e-5 / 1e9
+        assert sel["achieved"] == pytest.approx(gbs) and sel["frac"] == pytest.approx(gbs / 6000.0)
+
+
+def test_traffic_is_null_once_the_sources_change(tmp_path, monkeypatch):
+    # a DRAM-bytes entry counts only while the attention path's sources hash to
+    # the value it was captured on
+    from h2o_kv_cache_b200.workload import CONFIGS
+    b = _bench()
+    csrc = tmp_path / "h2o_kv_cache_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for n in b.KERNEL_SOURCES["fused"]:
+        (csrc / n).write_text("// " + n + "\n")
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    cfg = CONFIGS[4]
+    (tmp_path / "profiles").mkdir()
+    entry = {cfg.name: {"path": "fused", "sources_sha": b.sources_sha(b.KERNEL_SOURCES["fused"]),
+                        "dram_bytes_per_launch": 123.0}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(entry))
+    assert b.traffic_for(cfg) == 123.0
+    (csrc / b.KERNEL_SOURCES["fused"][0]).write_text("// changed\n")
+    assert b.traffic_for(cfg) is None
+
+
+def test_committed_traffic_entries_name_known_paths():
+    b = _bench()
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        entries = json.load(f)
+    for name, ent in entries.items():
+        assert ent["path"] in b.KERNEL_SOURCES, name
+        assert ent["dram_bytes_per_launch"] > 0, name
+        assert os.path.exists(os.path.join(ROOT, ent["source"])), name
